@@ -1,0 +1,417 @@
+#!/usr/bin/env python3
+"""Benchmark of the SmoothQuant W8A8 smoothed linear layer on B200.
+
+One step = one pass of the whole path over one batch of the 7B-like QKV
+projection prefill workload (X bf16 [4096 x 4096] with 0.1% outlier channels,
+W bf16 [12288 x 4096], alpha 0.5, bf16 output):
+  a1 calibrate X and W -> a2 smoothing factors -> a3 fold + quantize W ->
+  a4 smooth + quantize X -> a5 int8 GEMM with dequant epilogue,
+each a call into libsq's C ABI on one CUDA stream. L2 is flushed between
+steps; every kernel is bracketed by CUDA events on that stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs an independent
+replica (the path has no exchange step); value = all ranks' work / the slowest
+rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w8a8_post_quantization_calibrate_b200 import synth  # noqa: E402
+
+METRIC = "W8A8 smoothed-linear int8 TOPS & act-quant GB/s at 1 B200; % of roofline"
+WORKLOAD = "qkv_prefill_7b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOP/s bf16)
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+GEMM_SOURCES = ["w8a8_post_quantization_calibrate_b200/csrc/sq_gemm.cu",
+                "w8a8_post_quantization_calibrate_b200/csrc/sq_device.cuh"]
+
+
+def gemm_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when
+    absent or taken on a different version of the kernel source."""
+    p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_sha256_16") != gemm_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML while the
+    timed region runs (reads only; changes no setting)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self.err = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.nvml = None
+            self.err = repr(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                sm = self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+                util = self.nvml.nvmlDeviceGetUtilizationRates(self.h).gpu
+                reasons = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = self.nvml.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((sm, util, reasons, pw))
+            except Exception as e:  # pragma: no cover
+                self.err = repr(e)
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.nvml is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": self.err or "no samples"}
+        loaded = [s for s in self.samples if s[1] > 0] or self.samples
+        seen = 0
+        for s in loaded:
+            seen |= s[2]
+        reasons = [name for bit, name in self.REASONS.items() if seen & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(loaded),
+                "power_w_max": round(max(s[3] for s in loaded), 1)}
+
+
+# ------------------------------------------------------------------ the CPU oracle
+def oracle_sample(x: torch.Tensor, w: torch.Tensor, alpha: float, seconds: float,
+                  tokens: int = 64, rows: int = 256):
+    """The oracle, as it stands, on a bounded sample of the workload: the whole
+    path on a slice of `tokens` tokens x `rows` output channels (full K),
+    repeated until `seconds` have passed. Returns (TOPS, threads, description,
+    seconds per slice)."""
+    import oracle
+    hx = synth.host_array(x[:tokens])
+    hw = synth.host_array(w[:rows])
+    K = x.shape[1]
+    ops = 2.0 * tokens * rows * K
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.linear(hx, hw, alpha)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    per = el / n
+    desc = (f"whole path (a1..a5) on a {tokens}-token x {rows}-output-channel slice of the workload "
+            f"(K={K}), {n} repetitions in {el:.1f} s; value = 2*{tokens}*{rows}*{K} int8 ops per slice / time")
+    return ops / per / 1e12, oracle.num_threads(), desc, per
+
+
+# ------------------------------------------------------------------ our arm
+def kernel_bytes(M, N, K, in_es, out_es):
+    """Algorithmic bytes per launch of each step (reads + writes, each tensor once)."""
+    return {
+        "a1_calibrate_x": M * K * in_es + K * 4,
+        "a1_calibrate_w": N * K * in_es + K * 4,
+        "a2_smooth_factors": 3 * K * 4,
+        "a3_fold_quant_w": N * K * in_es + K * 4 + N * K + N * 4,
+        "a4_smooth_quant_x": M * K * in_es + K * 4 + M * K + M * 4,
+        "a5_w8a8_gemm": M * K + N * K + M * 4 + N * 4 + M * N * out_es,
+    }
+
+
+def run_ours(args, world, rank, local):
+    from w8a8_post_quantization_calibrate_b200 import sq
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    wl = synth.WORKLOADS[WORKLOAD]
+    M, N, K = wl.T, wl.N, wl.K
+    x_cpu, w_cpu = synth.make(WORKLOAD)
+    x = x_cpu.to(dev)
+    w = w_cpu.to(dev)
+    in_es, out_es = 2, 2
+    stream = torch.cuda.current_stream(dev)
+
+    xmax = torch.zeros(K, dtype=torch.float32, device=dev)
+    wmax = torch.zeros(K, dtype=torch.float32, device=dev)
+    maxima = torch.cat([xmax, wmax])  # one buffer, cleared once per step
+    xmax, wmax = maxima[:K], maxima[K:]
+    s = torch.empty(K, dtype=torch.float32, device=dev)
+    wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+    wsc = torch.empty(N, dtype=torch.float32, device=dev)
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    xsc = torch.empty(M, dtype=torch.float32, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    gws = sq.gemm_workspace(M, N, K, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    names = ["a1_calibrate_x", "a1_calibrate_w", "a2_smooth_factors", "a3_fold_quant_w",
+             "a4_smooth_quant_x", "a5_w8a8_gemm"]
+    launches_per_step = len(names)
+
+    def step(ev=None):
+        maxima.zero_()
+        if ev: ev[0].record(stream)
+        sq.sq_calibrate_absmax(x, xmax, stream=stream)
+        if ev: ev[1].record(stream)
+        sq.sq_calibrate_absmax(w, wmax, stream=stream)
+        if ev: ev[2].record(stream)
+        sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream)
+        if ev: ev[3].record(stream)
+        sq.sq_fold_quant_weights(w, s, wq=wq, w_scale=wsc, stream=stream)
+        if ev: ev[4].record(stream)
+        sq.sq_smooth_quant_act(x, s, xq=xq, x_scale=xsc, stream=stream)
+        if ev: ev[5].record(stream)
+        sq.sq_w8a8_gemm(xq, xsc, wq, wsc, y=y, workspace=gws, stream=stream)
+        if ev: ev[6].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if sq.sq_get_status(stream) != sq.SQ_OK:
+        raise RuntimeError("device status error during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(events[i])
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    status = sq.sq_get_status(stream)
+    if status != sq.SQ_OK:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    per_kernel = {n: 0.0 for n in names}
+    step_ms = 0.0
+    for ev in events:
+        step_ms += ev[0].elapsed_time(ev[6])
+        for j, n in enumerate(names):
+            per_kernel[n] += ev[j].elapsed_time(ev[j + 1])
+    step_ms /= args.steps
+    per_kernel = {n: v / args.steps for n, v in per_kernel.items()}
+    step_ms_max = max_over_ranks(step_ms, world, dev)
+    ops = 2.0 * M * N * K
+    value = world * ops / (step_ms_max * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    int8_peak = bf16_peak * INT8_OVER_BF16
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    kb = kernel_bytes(M, N, K, in_es, out_es)
+    kernels = {}
+    for n in names:
+        ms = per_kernel[n]
+        entry = {"ms": round(ms, 5), "gbs": round(kb[n] / (ms * 1e-3) / 1e9, 1),
+                 "hbm_frac": round(kb[n] / (ms * 1e-3) / 1e9 / hbm, 3)}
+        if n == "a5_w8a8_gemm":
+            tops = ops / (ms * 1e-3) / 1e12
+            entry.update({"tops": round(tops, 1), "tensor_frac": round(tops / int8_peak, 3)})
+        kernels[n] = entry
+    gemm_ms = per_kernel["a5_w8a8_gemm"]
+    achieved = ops / (gemm_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "gemm_tiled_kernel (a5)", "achieved": round(achieved, 1),
+                "peak": round(int8_peak, 1), "unit": "TOPS", "frac": round(achieved / int8_peak, 4),
+                "traffic": load_traffic(),
+                "peak_source": f"{peak_src}: bf16 {bf16_peak} TFLOP/s (burst) x {INT8_OVER_BF16} nominal "
+                               f"int8/bf16 ratio",
+                "algorithmic_ops_per_launch": ops}
+
+    # end to end through the public API: pinned host X and W in, host Y out
+    e2e = None
+    if args.e2e_steps > 0:
+        xh = x_cpu.pin_memory()
+        wh = w_cpu.pin_memory()
+        yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        lws = torch.zeros(sq.sq_linear_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            sq.sq_linear(xh, wh, wl.alpha, y=yh, workspace=lws, stream=stream)
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.e2e_steps)]
+        barrier(world)
+        for a, b in ev:
+            a.record(stream)
+            sq.sq_linear(xh, wh, wl.alpha, y=yh, workspace=lws, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / len(ev), world, dev)
+        e2e = {"value": round(world * ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TOPS",
+               "ms_per_step": round(e2e_ms, 3),
+               "h2d_bytes_per_step": x_cpu.numel() * in_es + w_cpu.numel() * in_es,
+               "d2h_bytes_per_step": M * N * out_es,
+               "api": "sq_linear (C ABI) with pinned host buffers"}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        v, cores, desc, _ = oracle_sample(x_cpu, w_cpu, wl.alpha, args.cpu_seconds)
+        cpu_baseline = {"value": round(v, 5), "unit": "TOPS", "cores": cores, "kind": "oracle",
+                        "sample": desc}
+
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded outlier-bearing activations, N(0,1/64) weights)",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "in_dtype": "bf16", "out_dtype": "bf16",
+                   "alpha": wl.alpha, "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "step": "a1(X) a1(W) a2 a3 a4 a5, one stream"},
+        "act_quant_gbs": kernels["a4_smooth_quant_x"]["gbs"],
+        "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu_baseline, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
+    }
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, world, rank):
+    """The oracle (plain C on the host cores) on this workload, as the
+    reference arm: each step is one bounded sample of the workload."""
+    if rank != 0:
+        return None
+    wl = synth.WORKLOADS[WORKLOAD]
+    x_cpu, w_cpu = synth.make(WORKLOAD)
+    budget = max(0.002, args.reference_budget_s / max(1, args.steps + args.warmup))
+    # size the slice so one step stays within the budget
+    tokens, rows = 64, 256
+    _, _, _, per = oracle_sample(x_cpu, w_cpu, wl.alpha, 0.0, tokens, rows)
+    while per > budget and tokens > 1:
+        tokens //= 2
+        per /= 2
+    for _ in range(args.warmup):
+        oracle_sample(x_cpu, w_cpu, wl.alpha, 0.0, tokens, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(x_cpu, w_cpu, wl.alpha, 0.0, tokens, rows)
+    el = time.perf_counter() - t0
+    ops = 2.0 * tokens * rows * wl.K
+    value = ops * args.steps / el / 1e12
+    import oracle
+    desc = (f"oracle whole path (a1..a5) on a {tokens}-token x {rows}-output-channel slice of the "
+            f"workload per step (K={wl.K}); value = int8 ops of the slice / time")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "M": wl.T, "N": wl.N, "K": wl.K,
+                                        "in_dtype": "bf16", "out_dtype": "bf16", "alpha": wl.alpha},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10, help="steps of the end-to-end measurement")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
+    ap.add_argument("--reference-budget-s", type=float, default=90.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if world != args.gpus and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        out = run_reference(args, world, rank)
+    else:
+        out = run_ours(args, world, rank, local)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

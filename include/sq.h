@@ -1,0 +1,203 @@
+/*
+ * sq.h -- C ABI of libsq, the SmoothQuant W8A8 linear layer on NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer computes Y = X W^T with X [T x K] (tokens x input channels) and
+ * W [N x K] (output x input channels), summing over K ("One outlier"
+ * quantization notes, "Which scales factor out, and why"). SmoothQuant divides
+ * activation channel j by s_j and multiplies weight input column j by s_j, an
+ * exact rewrite X W^T = (X diag(s)^-1)(W diag(s))^T ("SmoothQuant Explained",
+ * "The transform"), then runs both operands through symmetric int8 and an
+ * integer GEMM whose epilogue applies one scale per token and one per output
+ * channel ("Why do activation outliers break INT8 W8A8 on LLMs...", "A strong
+ * answer").
+ *
+ * Conventions for every call
+ *  - Matrices are row-major with leading dimension equal to their column
+ *    count, and start on a 16-byte boundary. K (the column count of X and W)
+ *    must be a multiple of 16.
+ *  - Unless a call says otherwise, pointers are CUDA device memory owned by
+ *    the caller. The library never frees or keeps them.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream). A status of SQ_OK means the arguments were accepted and
+ *    the work was enqueued; a kernel-side failure (a bounded wait that ran
+ *    out) is reported later by sq_get_status().
+ *  - Calls allocate no device memory. sq_w8a8_gemm and sq_linear take a
+ *    caller-provided workspace sized by their *_workspace_size function.
+ *  - Outputs must not alias inputs.
+ *  - There is no CPU fallback: every step runs in this library's kernels.
+ *
+ * Rounding: round to nearest, ties to even, everywhere a value is rounded.
+ * int8 codes use the symmetric range [-127, 127] ("One outlier" notes, "The
+ * four operations").
+ */
+#ifndef SQ_H_
+#define SQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* sq_stream_t;
+
+typedef enum sq_status {
+    SQ_OK = 0,
+    SQ_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, alpha outside [0,1], eps < 0,
+                                workspace too small */
+    SQ_ERR_UNSUPPORTED = 2,  /* K not a multiple of 16, misaligned pointer, unsupported dtype
+                                or size */
+    SQ_ERR_CUDA = 3,         /* a CUDA runtime call failed; see sq_last_error_string() */
+    SQ_ERR_TIMEOUT = 4       /* a kernel's bounded wait ran out (reported by sq_get_status) */
+} sq_status;
+
+typedef enum sq_dtype {
+    SQ_F32 = 0,   /* IEEE binary32 */
+    SQ_BF16 = 1,  /* bfloat16 (top half of a binary32) */
+    SQ_I32 = 2    /* int32: raw GEMM accumulators (output only) */
+} sq_dtype;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int sq_version(void);
+
+/* ---------------------------------------------------------------- step a1
+ * Per-input-channel absolute maximum (calibration).
+ *   absmax[j] = max(absmax[j], max_r |x[r, j]|)
+ * Defined by the numerator and denominator maxima of the smoothing factor:
+ * max_t |X_tj| over tokens and max_n |W_nj| over output channels
+ * ("Why do activation outliers break INT8 W8A8...", "A strong answer"; "One
+ * outlier" notes, "Route it, or move it": amax over dim 0). Applied to X it
+ * calibrates activations; applied to W [N x K] it gives the weight maxima.
+ *   x       [rows x cols], dtype dt (SQ_F32 or SQ_BF16), device.
+ *   absmax  [cols] float, device, in/out: a running maximum. The caller sets it
+ *           to +0 before the first batch; repeated calls over calibration
+ *           batches accumulate (the pages warn that the calibration set must
+ *           contain the outlier channels' true maxima).
+ * cols must be a multiple of 16. rows == 0 is a no-op. NaN inputs are not
+ * supported. Exact (max is order-independent). */
+sq_status sq_calibrate_absmax(const void* x, sq_dtype dt, int64_t rows, int64_t cols,
+                              float* absmax, sq_stream_t stream);
+
+/* ---------------------------------------------------------------- step a2
+ * Smoothing factors
+ *   s_j = max(xmax_j, eps)^alpha / max(wmax_j, eps)^(1 - alpha)
+ * ("SmoothQuant Explained", "Alpha: how much difficulty to move"; the eps
+ * clamp of both maxima follows "One outlier" notes, "Route it, or move it").
+ * Evaluated in fp64 and rounded once to fp32. For alpha in {0, 1/4, 1/2, 3/4, 1}
+ * the powers are exact compositions of correctly rounded sqrt, so the result
+ * is reproducible bit for bit; other alphas use pow() (within 1 fp32 ulp of
+ * the exact value).
+ *   xmax, wmax [K] float, device.   s [K] float, device, out.
+ *   alpha in [0, 1], eps >= 0 (1e-8 in the pages). */
+sq_status sq_smooth_factors(const float* xmax, const float* wmax, int64_t K, float alpha,
+                            float eps, float* s, sq_stream_t stream);
+
+/* ---------------------------------------------------------------- step a3
+ * Fold s into the weights and quantize per output channel.
+ *   What_nj   = W_nj * s_j                              (fp32)
+ *   w_scale_n = max_j |What_nj| / 127                   (1.0 for an all-zero row)
+ *   wq_nj     = clamp(round(What_nj / w_scale_n), -127, 127)
+ * ("Why do activation outliers break INT8 W8A8...", "A strong answer": the
+ * weight columns absorb s_j before quantization, per-output-channel scales;
+ * "One outlier" notes, "The four operations" for the quantizer and the
+ * zero-range case.)
+ *   w        [N x K], dtype dt (SQ_F32 or SQ_BF16), device.
+ *   s        [K] float, device.
+ *   wq       [N x K] int8, device, out.
+ *   w_scale  [N] float, device, out. */
+sq_status sq_fold_quant_weights(const void* w, sq_dtype dt, int64_t N, int64_t K,
+                                const float* s, int8_t* wq, float* w_scale,
+                                sq_stream_t stream);
+
+/* ---------------------------------------------------------------- step a4
+ * Smooth the activations and quantize per token (dynamic scale).
+ *   Xhat_tj   = X_tj / s_j                              (fp32 division)
+ *   x_scale_t = max_j |Xhat_tj| / 127                   (1.0 for an all-zero row)
+ *   xq_tj     = clamp(round(Xhat_tj / x_scale_t), -127, 127)
+ * ("SmoothQuant Explained", "The transform" and O1 per-token dynamic
+ * quantization in "Where it fits"; "Why are activations harder to quantize...",
+ * "Dynamic scaling".)
+ *   x        [T x K], dtype dt (SQ_F32 or SQ_BF16), device.
+ *   s        [K] float, device.
+ *   xq       [T x K] int8, device, out.
+ *   x_scale  [T] float, device, out. */
+sq_status sq_smooth_quant_act(const void* x, sq_dtype dt, int64_t T, int64_t K,
+                              const float* s, int8_t* xq, float* x_scale,
+                              sq_stream_t stream);
+
+/* ---------------------------------------------------------------- step a5
+ * int8 x int8 -> int32 GEMM with the dequantizing epilogue.
+ *   acc_tn = sum_k xq_tk * wq_nk                        (exact int32)
+ *   y_tn   = (float(acc_tn) * x_scale_t) * w_scale_n    (two fp32 roundings)
+ * ("Activation Outlier Channels and Mixed-Precision Decomposition",
+ * "Decomposition": integer matmul, float epilogue; "One outlier" notes, "Which
+ * scales factor out, and why": per-token and per-output-channel scales leave
+ * the integer sum untouched.)
+ *   xq [M x K] int8, x_scale [M] float, wq [N x K] int8, w_scale [N] float: device.
+ *   y  [M x N], out_dt = SQ_BF16 (fp32 value rounded to nearest even), SQ_F32, or
+ *      SQ_I32 (the raw accumulators; scales ignored and may be NULL).
+ *   workspace: device, ws_bytes >= sq_w8a8_gemm_workspace_size(M, N, K). When the
+ *      required size is non-zero (small M, the split-K weight-streaming path) the
+ *      workspace must be zero-filled before its first use; every call that
+ *      completes leaves it zero-filled again. Calls that share a workspace must
+ *      not overlap on the GPU.
+ * |acc| <= 127 * 127 * K, which fits int32 for every K <= 133,144; larger K is
+ * rejected (SQ_ERR_UNSUPPORTED). */
+size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+sq_status sq_w8a8_gemm(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                       const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
+                       sq_dtype out_dt, void* workspace, size_t ws_bytes,
+                       sq_stream_t stream);
+
+/* ---------------------------------------------------------------- whole layer
+ * The whole path on one batch: calibrate X and W (a1, from zero), smoothing
+ * factors (a2), fold + quantize W (a3), smooth + quantize X (a4), GEMM with
+ * dequant (a5).
+ *   x [M x K], w [N x K]: dtype in_dt (SQ_F32 or SQ_BF16).
+ *   y [M x N]: dtype out_dt (SQ_F32 or SQ_BF16).
+ *   x, w and y may each be device memory or host memory (pinned host memory
+ *   copies asynchronously; pageable host memory makes the copy synchronous).
+ *   Host operands are staged through the workspace with cudaMemcpyAsync on
+ *   `stream`; for a host y the call returns before the copy-back completes, so
+ *   synchronize `stream` before reading it.
+ *   workspace: device, ws_bytes >= sq_linear_workspace_size(...); it holds the
+ *   maxima, factors, codes, scales and (for host operands) the staged copies.
+ *   Zero-fill it once before its first use (it contains the GEMM workspace). */
+size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K, sq_dtype in_dt,
+                                sq_dtype out_dt);
+sq_status sq_linear(const void* x, const void* w, sq_dtype in_dt, int64_t M, int64_t N,
+                    int64_t K, float alpha, float eps, void* y, sq_dtype out_dt,
+                    void* workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* ---------------------------------------------------------------- status
+ * Synchronize `stream`, then return and clear the first error any kernel of
+ * this library recorded on the current device since the last call (SQ_OK if
+ * none). SQ_ERR_TIMEOUT means a bounded wait inside a kernel ran out; the
+ * kernel stopped and the CUDA context stays usable. */
+sq_status sq_get_status(sq_stream_t stream);
+
+/* Site code of the error sq_get_status() last returned (0 if none). */
+unsigned int sq_last_status_site(void);
+
+/* Human-readable description of the last host-side error on this thread. */
+const char* sq_last_error_string(void);
+
+/* Limit, in milliseconds, for every bounded wait inside the kernels (default
+ * 2000). Applies to launches made after the call, on every device. */
+sq_status sq_set_wait_timeout_ms(int64_t ms);
+
+/* Self-test of the bounded-wait machinery: launches one CTA that waits, with a
+ * limit of `limit_us` microseconds, on a barrier that nothing arrives at. The
+ * wait runs out, the kernel records SQ_ERR_TIMEOUT and returns. Used by tests
+ * to show that a stalled wait ends with a status instead of a hang. */
+sq_status sq_selftest_wait_timeout(int64_t limit_us, sq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H_ */

@@ -1,0 +1,663 @@
+// sq_gemm.cu -- step a5: int8 x int8 -> int32 GEMM with the dequantizing
+// epilogue, on the sm_100a tensor cores (tcgen05.mma kind::i8, TMEM int32
+// accumulators, TMA-fed 128B-swizzled shared-memory tiles).
+//
+//   acc[t, n] = sum_k xq[t, k] * wq[n, k]
+//   y[t, n]   = (float(acc[t, n]) * x_scale[t]) * w_scale[n]
+//
+// Per-token and per-output-channel scales are constant along K, so they leave
+// the integer sum untouched and are applied once, after it ("One outlier"
+// notes, "Which scales factor out, and why"; "Activation Outlier Channels and
+// Mixed-Precision Decomposition", "Decomposition": integer matmul, float
+// epilogue).
+//
+// Two kernels:
+//  * gemm_tiled_kernel (prefill, M > 16): persistent CTAs, one per SM, over
+//    128 x 256 output tiles. Warp 0 streams A/B k-blocks with TMA into a
+//    4-stage ring; one thread of warp 1 issues tcgen05.mma (M=128, N=256,
+//    K=32) into one of two TMEM accumulators; warps 2-5 drain the other
+//    accumulator (tcgen05.ld), apply the scales and store Y, overlapping the
+//    next tile's main loop.
+//  * gemm_stream_kernel (decode, M <= 16): the product is computed transposed,
+//    Y^T = Wq Xq^T, so the weight rows fill the 128-row MMA side and the few
+//    tokens are the N=16 side. The weight matrix is streamed once from HBM,
+//    split over all SMs along (row tile, k-block) work units; partial int32
+//    sums of a row tile meet in a global workspace (exact integer atomics) and
+//    the CTA that completes a tile applies the epilogue and re-zeroes it.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "sq_device.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+
+// ------------------------------------------------------------------ shapes
+constexpr int BM = 128;          // output rows per tile (tokens)
+constexpr int BN = 256;          // output columns per tile (output channels)
+constexpr int BK = 128;          // k-block: 128 int8 = one 128-byte swizzle row
+constexpr int UMMA_K = 32;       // K of one kind::i8 MMA
+constexpr int STAGES = 4;
+constexpr uint32_t A_STAGE = BM * BK;           // 16 KB
+constexpr uint32_t B_STAGE = BN * BK;           // 32 KB
+constexpr int ACC_COLS = BN;                    // int32 columns per accumulator
+constexpr int TMEM_COLS = 2 * ACC_COLS;         // double-buffered: 512 columns
+constexpr int GEMM_THREADS = 192;               // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr uint32_t IDESC_TILED = make_idesc_i8(BM, BN);
+
+constexpr int S_BM = 128;        // weight rows per tile (MMA M)
+constexpr int S_BN = 16;         // tokens (MMA N)
+constexpr int S_STAGES = 8;
+constexpr uint32_t S_A_STAGE = S_BM * BK;       // 16 KB
+constexpr uint32_t S_B_STAGE = S_BN * BK;       // 2 KB
+constexpr int S_TMEM_COLS = 32;                 // 2 x 16 columns
+constexpr uint32_t IDESC_STREAM = make_idesc_i8(S_BM, S_BN);
+constexpr int STREAM_MAX_M = 16;
+
+enum OutKind { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
+
+constexpr size_t tiled_smem_bytes() {
+    return 1024 /*alignment slack*/ + STAGES * (A_STAGE + B_STAGE) + 256 /*barriers etc*/;
+}
+constexpr size_t stream_smem_bytes() {
+    return 1024 + S_STAGES * (S_A_STAGE + S_B_STAGE) + 256;
+}
+
+// Tile order: groups of 16 row tiles, column tiles outermost inside a group, so
+// the CTAs in flight at one time share few A and B panels (L2 reuse).
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
+    constexpr int GROUP = 16;
+    const int group = tile / (GROUP * num_n);
+    const int first_m = group * GROUP;
+    const int gm = min(num_m - first_m, GROUP);
+    const int idx = tile - group * GROUP * num_n;
+    mb = first_m + idx % gm;
+    nb = idx / gm;
+}
+
+// Stores 32 consecutive outputs of one row (row-major y, row stride N).
+template <int OUT>
+__device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int N, const uint32_t (&r)[32],
+                                            float sa, const float* __restrict__ w_scale) {
+    const int64_t base = row * (int64_t)N + col0;
+    const bool full = (col0 + 32 <= N);
+    if (OUT == kOutI32) {
+        int32_t* yp = static_cast<int32_t*>(y) + base;
+        if (full && (N & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<int4*>(yp + i) = make_int4((int)r[i], (int)r[i + 1], (int)r[i + 2], (int)r[i + 3]);
+        } else {
+            for (int i = 0; i < 32; ++i)
+                if (col0 + i < N) yp[i] = (int32_t)r[i];
+        }
+        return;
+    }
+    float v[32];
+    if (full) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+            const float4 sw = __ldg(reinterpret_cast<const float4*>(w_scale + col0 + i));
+            v[i] = dequant((int32_t)r[i], sa, sw.x);
+            v[i + 1] = dequant((int32_t)r[i + 1], sa, sw.y);
+            v[i + 2] = dequant((int32_t)r[i + 2], sa, sw.z);
+            v[i + 3] = dequant((int32_t)r[i + 3], sa, sw.w);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            v[i] = (col0 + i < N) ? dequant((int32_t)r[i], sa, __ldg(w_scale + col0 + i)) : 0.0f;
+    }
+    if (OUT == kOutF32) {
+        float* yp = static_cast<float*>(y) + base;
+        if (full && (N & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(yp + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        } else {
+            for (int i = 0; i < 32; ++i)
+                if (col0 + i < N) yp[i] = v[i];
+        }
+    } else {
+        __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(y) + base;
+        if (full && (N & 7) == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+                uint4 pk;
+                pk.x = pack_bf16x2(v[i], v[i + 1]);
+                pk.y = pack_bf16x2(v[i + 2], v[i + 3]);
+                pk.z = pack_bf16x2(v[i + 4], v[i + 5]);
+                pk.w = pack_bf16x2(v[i + 6], v[i + 7]);
+                *reinterpret_cast<uint4*>(yp + i) = pk;
+            }
+        } else {
+            for (int i = 0; i < 32; ++i)
+                if (col0 + i < N) yp[i] = __float2bfloat16_rn(v[i]);
+        }
+    }
+}
+
+// ================================================================== prefill
+template <int OUT>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const float* __restrict__ x_scale, const float* __restrict__ w_scale,
+                  void* __restrict__ y, int M, int N, int K, long long wait_limit) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * A_STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+    // bars: full[STAGES] | empty[STAGES] | tfull[2] | tempty[2] | drain
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    __shared__ int no_abort;  // always 0: drain waits must not be cut short by the abort flag
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int num_kb = (K + BK - 1) / BK;
+
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+    const int FULL = 0, EMPTY = STAGES, TFULL = 2 * STAGES, TEMPTY = 2 * STAGES + 2, DRAIN = 2 * STAGES + 4;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar(FULL + s), 1);
+            mbar_init(bar(EMPTY + s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar(TFULL + a), 1);
+            mbar_init(bar(TEMPTY + a), 4);
+        }
+        mbar_init(bar(DRAIN), 1);
+        *abort_flag = 0;
+        no_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc<TMEM_COLS>(smem_u32(tmem_holder));
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                int mb, nb;
+                tile_coords(tile, num_m, num_n, mb, nb);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar(EMPTY + stage), phase ^ 1, wait_limit, abort_flag, SITE_GEMM_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar(FULL + stage), A_STAGE + B_STAGE);
+                    tma_load_2d(smem_u32(sA + stage * A_STAGE), &tmA, bar(FULL + stage), kb * BK, mb * BM);
+                    tma_load_2d(smem_u32(sB + stage * B_STAGE), &tmB, bar(FULL + stage), kb * BK, nb * BN);
+                    ++issued;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok || *abort_flag) {
+                // Every bulk copy this CTA started must land before the CTA exits.
+                for (int s = 0; s < STAGES; ++s) {
+                    const long long cnt = issued / STAGES + (s < issued % STAGES ? 1 : 0);
+                    if (cnt > 0)
+                        mbar_wait(bar(FULL + s), (uint32_t)((cnt - 1) & 1), wait_limit, &no_abort, SITE_GEMM_DRAIN);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!mbar_wait(bar(TEMPTY + acc), acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM_MMA_TMEM)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar(FULL + stage), phase, wait_limit, abort_flag, SITE_GEMM_MMA_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
+                    const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k)
+                        mma_i8(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
+                               make_sw128_kmajor_desc(b0 + k * UMMA_K), IDESC_TILED,
+                               (kb | k) != 0 ? 1u : 0u);
+                    mma_commit(bar(EMPTY + stage));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(bar(TFULL + acc));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            // All issued MMAs must finish before TMEM is released.
+            mma_commit(bar(DRAIN));
+            mbar_wait(bar(DRAIN), 0, wait_limit, &no_abort, SITE_GEMM_DRAIN);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (warps 2..5)
+        const int quarter = warp & 3;  // TMEM lanes this warp may read: 32*quarter ..
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            if (!mbar_wait(bar(TFULL + acc), acc_phase, wait_limit, abort_flag, SITE_GEMM_EPILOGUE)) break;
+            tc_fence_after();
+            const int64_t row = (int64_t)mb * BM + quarter * 32 + lane;
+            const bool row_ok = row < M;
+            const float sa = (OUT != kOutI32 && row_ok) ? __ldg(x_scale + row) : 0.0f;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; c += 2) {
+                uint32_t r0[32], r1[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, r0);
+                tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
+                tmem_wait_ld();
+                const int col0 = nb * BN + c * 32;
+                if (row_ok && col0 < N) store_row32<OUT>(y, row, col0, N, r0, sa, w_scale);
+                if (row_ok && col0 + 32 < N) store_row32<OUT>(y, row, col0 + 32, N, r1, sa, w_scale);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(TEMPTY + acc));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc<TMEM_COLS>(tmem_base);
+    }
+}
+
+// ================================================================== decode
+// Work unit = (row tile of W, k-block). CTA c owns units [c*U/G, (c+1)*U/G);
+// a maximal run of its units inside one row tile is a segment, accumulated in
+// TMEM and added into ws_acc[t * N + n] with integer atomics. tile_count[tile]
+// (one counter per 32-row quarter of the tile) counts k-blocks merged so far;
+// the warp that brings it to num_kb writes those rows of Y and leaves ws_acc /
+// tile_count zero again.
+template <int OUT>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                   const float* __restrict__ x_scale, const float* __restrict__ w_scale,
+                   void* __restrict__ y, int M, int N, int K,
+                   int32_t* __restrict__ ws_acc, unsigned int* __restrict__ tile_count,
+                   long long wait_limit) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + S_STAGES * S_A_STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S_STAGES * S_B_STAGE);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * S_STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    __shared__ int no_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = (N + S_BM - 1) / S_BM;
+    const int num_kb = (K + BK - 1) / BK;
+    const long long units = (long long)num_tiles * num_kb;
+    const long long u_begin = units * blockIdx.x / gridDim.x;
+    const long long u_end = units * (blockIdx.x + 1) / gridDim.x;
+
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+    const int FULL = 0, EMPTY = S_STAGES, TFULL = 2 * S_STAGES, TEMPTY = 2 * S_STAGES + 2, DRAIN = 2 * S_STAGES + 4;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S_STAGES; ++s) {
+            mbar_init(bar(FULL + s), 1);
+            mbar_init(bar(EMPTY + s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar(TFULL + a), 1);
+            mbar_init(bar(TEMPTY + a), 4);
+        }
+        mbar_init(bar(DRAIN), 1);
+        *abort_flag = 0;
+        no_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc<S_TMEM_COLS>(smem_u32(tmem_holder));
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (long long u = u_begin; u < u_end && ok; ++u) {
+                const int tile = (int)(u / num_kb), kb = (int)(u % num_kb);
+                if (!mbar_wait(bar(EMPTY + stage), phase ^ 1, wait_limit, abort_flag, SITE_STREAM_PRODUCER)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(bar(FULL + stage), S_A_STAGE + S_B_STAGE);
+                tma_load_2d(smem_u32(sA + stage * S_A_STAGE), &tmW, bar(FULL + stage), kb * BK, tile * S_BM);
+                tma_load_2d(smem_u32(sB + stage * S_B_STAGE), &tmX, bar(FULL + stage), kb * BK, 0);
+                ++issued;
+                if (++stage == S_STAGES) { stage = 0; phase ^= 1; }
+            }
+            if (!ok || *abort_flag) {
+                for (int s = 0; s < S_STAGES; ++s) {
+                    const long long cnt = issued / S_STAGES + (s < issued % S_STAGES ? 1 : 0);
+                    if (cnt > 0)
+                        mbar_wait(bar(FULL + s), (uint32_t)((cnt - 1) & 1), wait_limit, &no_abort, SITE_STREAM_DRAIN);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            long long u = u_begin;
+            while (u < u_end && ok) {
+                const int tile = (int)(u / num_kb);
+                const long long seg_end = min(u_end, (long long)(tile + 1) * num_kb);
+                if (!mbar_wait(bar(TEMPTY + acc), acc_phase ^ 1, wait_limit, abort_flag, SITE_STREAM_MMA_TMEM)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S_BN);
+                bool first = true;
+                for (; u < seg_end; ++u) {
+                    if (!mbar_wait(bar(FULL + stage), phase, wait_limit, abort_flag, SITE_STREAM_MMA_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * S_A_STAGE);
+                    const uint32_t b0 = smem_u32(sB + stage * S_B_STAGE);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        mma_i8(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
+                               make_sw128_kmajor_desc(b0 + k * UMMA_K), IDESC_STREAM,
+                               (first && k == 0) ? 0u : 1u);
+                    }
+                    first = false;
+                    mma_commit(bar(EMPTY + stage));
+                    if (++stage == S_STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(bar(TFULL + acc));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            mma_commit(bar(DRAIN));
+            mbar_wait(bar(DRAIN), 0, wait_limit, &no_abort, SITE_STREAM_DRAIN);
+        }
+        __syncwarp();
+    } else {
+        // Each epilogue warp owns 32 weight rows of the tile (its TMEM lane
+        // quarter) and its own completion counter, so no cross-warp barrier is
+        // needed and an aborted wait cannot strand the other warps.
+        const int quarter = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        long long u = u_begin;
+        while (u < u_end) {
+            const int tile = (int)(u / num_kb);
+            const long long seg_end = min(u_end, (long long)(tile + 1) * num_kb);
+            const unsigned int seg_len = (unsigned int)(seg_end - u);
+            u = seg_end;
+            if (!mbar_wait(bar(TFULL + acc), acc_phase, wait_limit, abort_flag, SITE_STREAM_EPILOGUE)) break;
+            tc_fence_after();
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * S_BN), r);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(TEMPTY + acc));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+
+            const int n = tile * S_BM + quarter * 32 + lane;
+            if (n < N) {
+#pragma unroll
+                for (int t = 0; t < S_BN; ++t)
+                    if (t < M) atomicAdd(ws_acc + (int64_t)t * N + n, (int32_t)r[t]);
+            }
+            __threadfence();
+            __syncwarp();
+            unsigned int* cnt = tile_count + tile * 4 + quarter;
+            unsigned int prev = 0;
+            if (lane == 0) prev = atomicAdd(cnt, seg_len);
+            prev = __shfl_sync(0xffffffffu, prev, 0);
+            if (prev + seg_len == (unsigned int)num_kb) {
+                // Last contributor of these 32 rows: every other CTA's partial
+                // sums are in ws_acc. Write Y and leave the workspace zeroed.
+                __threadfence();
+                if (n < N) {
+                    const float sw = (OUT != kOutI32) ? __ldg(w_scale + n) : 0.0f;
+                    for (int t = 0; t < M; ++t) {
+                        int32_t* p = ws_acc + (int64_t)t * N + n;
+                        const int32_t a = __ldcg(p);
+                        *p = 0;
+                        const int64_t o = (int64_t)t * N + n;
+                        if (OUT == kOutI32) {
+                            static_cast<int32_t*>(y)[o] = a;
+                        } else {
+                            const float v = dequant(a, __ldg(x_scale + t), sw);
+                            if (OUT == kOutF32) static_cast<float*>(y)[o] = v;
+                            else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) *cnt = 0u;
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc<S_TMEM_COLS>(tmem_base);
+    }
+}
+
+// ================================================================== host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+sq_status get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) {
+        set_error("cuTensorMapEncodeTiled is not available from the driver");
+        return SQ_ERR_CUDA;
+    }
+    return SQ_OK;
+}
+
+// Row-major int8 matrix [rows x K] as a 2-D tensor map with 128B swizzle and a
+// (128 bytes of K) x box_rows box. Out-of-range rows/columns read as zero.
+sq_status make_map_i8(CUtensorMap* map, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
+    sq_status r = get_encoder();
+    if (r != SQ_OK) return r;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult cr = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d) for a %lld x %lld int8 matrix", (int)cr,
+                  (long long)rows, (long long)K);
+        return SQ_ERR_CUDA;
+    }
+    return SQ_OK;
+}
+
+template <typename Kern>
+sq_status ensure_smem_attr(Kern k, size_t bytes, bool& done) {
+    // Per device: the attribute is a property of the function on the current device.
+    static thread_local int last_dev = -1;
+    (void)last_dev;
+    if (done) return SQ_OK;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+    done = true;
+    return SQ_OK;
+}
+
+template <int OUT>
+sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
+                       int M, int N, int K, cudaStream_t st) {
+    static bool attr_done[64] = {};
+    const DeviceInfo& di = device_info();
+    const size_t smem = tiled_smem_bytes();
+    sq_status r = ensure_smem_attr(gemm_tiled_kernel<OUT>, smem, attr_done[di.device & 63]);
+    if (r != SQ_OK) return r;
+    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = tiles < di.sm_count ? tiles : di.sm_count;
+    gemm_tiled_kernel<OUT><<<grid, GEMM_THREADS, smem, st>>>(ta, tb, xs, wsc, y, M, N, K, wait_limit_cycles());
+    return check_launch("gemm_tiled_kernel");
+}
+
+template <int OUT>
+sq_status launch_stream(const CUtensorMap& tw, const CUtensorMap& tx, const float* xs, const float* wsc, void* y,
+                        int M, int N, int K, int32_t* ws_acc, unsigned int* counts, cudaStream_t st) {
+    static bool attr_done[64] = {};
+    const DeviceInfo& di = device_info();
+    const size_t smem = stream_smem_bytes();
+    sq_status r = ensure_smem_attr(gemm_stream_kernel<OUT>, smem, attr_done[di.device & 63]);
+    if (r != SQ_OK) return r;
+    const long long units = (long long)((N + S_BM - 1) / S_BM) * ((K + BK - 1) / BK);
+    const int grid = units < di.sm_count ? (int)units : di.sm_count;
+    gemm_stream_kernel<OUT><<<grid, GEMM_THREADS, smem, st>>>(tw, tx, xs, wsc, y, M, N, K, ws_acc, counts,
+                                                              wait_limit_cycles());
+    return check_launch("gemm_stream_kernel");
+}
+
+size_t stream_ws_bytes(int64_t M, int64_t N) {
+    const size_t acc = (size_t)M * (size_t)N * sizeof(int32_t);
+    const size_t acc_al = (acc + 255) & ~size_t(255);
+    const size_t cnt = (size_t)((N + S_BM - 1) / S_BM) * 4 * sizeof(unsigned int);
+    return acc_al + ((cnt + 255) & ~size_t(255));
+}
+
+}  // namespace
+
+size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+    (void)K;
+    if (M <= 0 || N <= 0) return 0;
+    return M <= STREAM_MAX_M ? stream_ws_bytes(M, N) : 0;
+}
+
+sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq, const float* w_scale,
+                        int64_t M, int64_t N, int64_t K, void* y, sq_dtype out_dt, void* workspace,
+                        size_t ws_bytes, cudaStream_t st) {
+    if (M < 0 || N < 0 || K < 0) { set_error("negative size"); return SQ_ERR_INVALID_ARG; }
+    if (out_dt != SQ_F32 && out_dt != SQ_BF16 && out_dt != SQ_I32) {
+        set_error("output dtype must be SQ_F32, SQ_BF16 or SQ_I32");
+        return SQ_ERR_UNSUPPORTED;
+    }
+    if (M == 0 || N == 0) return SQ_OK;
+    if (K == 0 || K % 16 != 0) { set_error("K=%lld must be a positive multiple of 16", (long long)K); return SQ_ERR_UNSUPPORTED; }
+    if (K > 133144) { set_error("K=%lld: 127*127*K would overflow int32", (long long)K); return SQ_ERR_UNSUPPORTED; }
+    if (M > 2147483647LL || N > 2147483647LL) { set_error("size too large"); return SQ_ERR_UNSUPPORTED; }
+    if (!xq || !wq || !y) { set_error("NULL pointer"); return SQ_ERR_INVALID_ARG; }
+    if (out_dt != SQ_I32 && (!x_scale || !w_scale)) { set_error("NULL scale pointer"); return SQ_ERR_INVALID_ARG; }
+    if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || (w_scale && !aligned16(w_scale))) {
+        set_error("xq, wq, y and w_scale must be 16-byte aligned");
+        return SQ_ERR_UNSUPPORTED;
+    }
+    const int out = out_dt == SQ_F32 ? kOutF32 : (out_dt == SQ_BF16 ? kOutBF16 : kOutI32);
+    sq_status r;
+    if (M <= STREAM_MAX_M) {
+        const size_t need = stream_ws_bytes(M, N);
+        if (!workspace || ws_bytes < need) {
+            set_error("workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+            return SQ_ERR_INVALID_ARG;
+        }
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+            set_error("workspace must be 256-byte aligned");
+            return SQ_ERR_UNSUPPORTED;
+        }
+        CUtensorMap tw, tx;
+        if ((r = make_map_i8(&tw, wq, N, K, S_BM)) != SQ_OK) return r;
+        if ((r = make_map_i8(&tx, xq, M, K, S_BN)) != SQ_OK) return r;
+        int32_t* ws_acc = static_cast<int32_t*>(workspace);
+        const size_t acc_al = (((size_t)M * N * 4) + 255) & ~size_t(255);
+        unsigned int* counts = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + acc_al);
+        switch (out) {
+            case kOutF32: return launch_stream<kOutF32>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, ws_acc, counts, st);
+            case kOutBF16: return launch_stream<kOutBF16>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, ws_acc, counts, st);
+            default: return launch_stream<kOutI32>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, ws_acc, counts, st);
+        }
+    }
+    CUtensorMap ta, tb;
+    if ((r = make_map_i8(&ta, xq, M, K, BM)) != SQ_OK) return r;
+    if ((r = make_map_i8(&tb, wq, N, K, BN)) != SQ_OK) return r;
+    switch (out) {
+        case kOutF32: return launch_tiled<kOutF32>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
+        case kOutBF16: return launch_tiled<kOutBF16>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
+        default: return launch_tiled<kOutI32>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
+    }
+}
+
+}  // namespace sq
+
+extern "C" {
+
+size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+    return sq::gemm_workspace_size(M, N, K);
+}
+
+sq_status sq_w8a8_gemm(const int8_t* xq, const float* x_scale, const int8_t* wq, const float* w_scale,
+                       int64_t M, int64_t N, int64_t K, void* y, sq_dtype out_dt, void* workspace,
+                       size_t ws_bytes, sq_stream_t stream) {
+    return sq::gemm_dispatch(xq, x_scale, wq, w_scale, M, N, K, y, out_dt, workspace, ws_bytes,
+                             (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// sq_internal.h -- host-side helpers shared by the library's translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "sq.h"
+
+namespace sq {
+
+// Thread-local last error message (sq_last_error_string).
+void set_error(const char* fmt, ...);
+
+// Record a CUDA runtime failure and return SQ_ERR_CUDA.
+sq_status cuda_fail(cudaError_t e, const char* what);
+
+// Check the last launch on this thread.
+inline sq_status check_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SQ_OK : cuda_fail(e, what);
+}
+
+// Device facts, cached per device.
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int clock_khz = 0;      // maximum SM clock
+    int max_smem_optin = 0; // bytes per block
+};
+const DeviceInfo& device_info();
+
+// Wait limit for bounded device waits, in SM clock cycles for the current device.
+long long wait_limit_cycles();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Site codes recorded with a device-side error (sq_last_status_site).
+enum Site : unsigned int {
+    SITE_SELFTEST = 1,
+    SITE_GEMM_PRODUCER = 10,
+    SITE_GEMM_MMA_FULL = 11,
+    SITE_GEMM_MMA_TMEM = 12,
+    SITE_GEMM_EPILOGUE = 13,
+    SITE_GEMM_DRAIN = 14,
+    SITE_STREAM_PRODUCER = 20,
+    SITE_STREAM_MMA_FULL = 21,
+    SITE_STREAM_MMA_TMEM = 22,
+    SITE_STREAM_EPILOGUE = 23,
+    SITE_STREAM_DRAIN = 24,
+};
+
+// Internal entry points used by sq_linear.
+sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                        const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
+                        sq_dtype out_dt, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+}  // namespace sq

@@ -1,0 +1,6 @@
+// sq_lib.cu -- libsq is compiled as one translation unit, so the device status
+// word defined in sq_api.cu is shared by every kernel without relocatable
+// device code.
+#include "sq_api.cu"
+#include "sq_quant.cu"
+#include "sq_gemm.cu"

@@ -1,0 +1,243 @@
+"""Thin Python binding of libsq (include/sq.h): argument marshalling only.
+
+Every function has the name of the C entry point it calls. Tensors are torch
+CUDA tensors (device memory and the current stream come from PyTorch); outputs
+not supplied by the caller are allocated with torch. All computation happens in
+libsq's kernels: importing this module loads libsq.so and raises if it has not
+been built -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsq.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "sq.h")
+
+SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
+SQ_F32, SQ_BF16, SQ_I32 = 0, 1, 2
+STATUS_NAMES = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED", 3: "SQ_ERR_CUDA",
+                4: "SQ_ERR_TIMEOUT"}
+
+
+class SqError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libsq.so is not built ({LIB_PATH}); run "
+                      "`python -m w8a8_post_quantization_calibrate_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i64, _f32, _sz, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_int
+
+_SIGS = {
+    "sq_version": ([], _int),
+    "sq_calibrate_absmax": ([_vp, _int, _i64, _i64, _vp, _vp], _int),
+    "sq_smooth_factors": ([_vp, _vp, _i64, _f32, _f32, _vp, _vp], _int),
+    "sq_fold_quant_weights": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "sq_smooth_quant_act": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "sq_w8a8_gemm_workspace_size": ([_i64, _i64, _i64], _sz),
+    "sq_w8a8_gemm": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp], _int),
+    "sq_linear_workspace_size": ([_i64, _i64, _i64, _int, _int], _sz),
+    "sq_linear": ([_vp, _vp, _int, _i64, _i64, _i64, _f32, _f32, _vp, _int, _vp, _sz, _vp], _int),
+    "sq_get_status": ([_vp], _int),
+    "sq_last_status_site": ([], ctypes.c_uint),
+    "sq_last_error_string": ([], ctypes.c_char_p),
+    "sq_set_wait_timeout_ms": ([_i64], _int),
+    "sq_selftest_wait_timeout": ([_i64, _vp], _int),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/sq.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(status: int, where: str) -> None:
+    if status != SQ_OK:
+        msg = _lib.sq_last_error_string().decode(errors="replace")
+        raise SqError(status, where, msg)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SQ_F32
+    if t.dtype == torch.bfloat16:
+        return SQ_BF16
+    if t.dtype == torch.int32:
+        return SQ_I32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _torch_dtype(code: int):
+    return {SQ_F32: torch.float32, SQ_BF16: torch.bfloat16, SQ_I32: torch.int32}[code]
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def sq_version() -> int:
+    return _lib.sq_version()
+
+
+def sq_calibrate_absmax(x: torch.Tensor, absmax: torch.Tensor, stream=None) -> torch.Tensor:
+    """Running per-column max |x| into `absmax` (float32 [cols], in/out)."""
+    rows, cols = x.shape
+    _check(_lib.sq_calibrate_absmax(_dev(x, "x"), _dt(x), rows, cols, _dev(absmax, "absmax"),
+                                    _stream(stream)), "sq_calibrate_absmax")
+    return absmax
+
+
+def sq_smooth_factors(xmax: torch.Tensor, wmax: torch.Tensor, alpha: float, eps: float = 1e-8,
+                      s: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    K = xmax.shape[0]
+    if s is None:
+        s = torch.empty(K, dtype=torch.float32, device=xmax.device)
+    _check(_lib.sq_smooth_factors(_dev(xmax, "xmax"), _dev(wmax, "wmax"), K, float(alpha), float(eps),
+                                  _dev(s, "s"), _stream(stream)), "sq_smooth_factors")
+    return s
+
+
+def sq_fold_quant_weights(w: torch.Tensor, s: torch.Tensor, wq: torch.Tensor | None = None,
+                          w_scale: torch.Tensor | None = None, stream=None):
+    N, K = w.shape
+    if wq is None:
+        wq = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=w.device)
+    _check(_lib.sq_fold_quant_weights(_dev(w, "w"), _dt(w), N, K, _dev(s, "s"), _dev(wq, "wq"),
+                                      _dev(w_scale, "w_scale"), _stream(stream)), "sq_fold_quant_weights")
+    return wq, w_scale
+
+
+def sq_smooth_quant_act(x: torch.Tensor, s: torch.Tensor, xq: torch.Tensor | None = None,
+                        x_scale: torch.Tensor | None = None, stream=None):
+    T, K = x.shape
+    if xq is None:
+        xq = torch.empty((T, K), dtype=torch.int8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(_lib.sq_smooth_quant_act(_dev(x, "x"), _dt(x), T, K, _dev(s, "s"), _dev(xq, "xq"),
+                                    _dev(x_scale, "x_scale"), _stream(stream)), "sq_smooth_quant_act")
+    return xq, x_scale
+
+
+def sq_w8a8_gemm_workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib.sq_w8a8_gemm_workspace_size(M, N, K))
+
+
+_ws_cache: dict = {}
+
+
+def gemm_workspace(M: int, N: int, K: int, device) -> torch.Tensor | None:
+    """A zero-filled workspace for sq_w8a8_gemm, cached per (device, size);
+    calls that complete leave it zero-filled, as the C API requires."""
+    need = sq_w8a8_gemm_workspace_size(M, N, K)
+    if need == 0:
+        return None
+    key = (str(device), need)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def sq_w8a8_gemm(xq: torch.Tensor, x_scale: torch.Tensor | None, wq: torch.Tensor,
+                 w_scale: torch.Tensor | None, out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    M, K = xq.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, xq.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.sq_w8a8_gemm(_dev(xq, "xq"), x_scale.data_ptr() if x_scale is not None else None,
+                             _dev(wq, "wq"), w_scale.data_ptr() if w_scale is not None else None,
+                             M, N, K, _dev(y, "y"), _dt(y), ws_ptr, ws_bytes, _stream(stream)),
+           "sq_w8a8_gemm")
+    return y
+
+
+def sq_linear_workspace_size(M: int, N: int, K: int, in_dtype=torch.bfloat16, out_dtype=torch.bfloat16) -> int:
+    return int(_lib.sq_linear_workspace_size(M, N, K, _dt(torch.empty(0, dtype=in_dtype)),
+                                             _dt(torch.empty(0, dtype=out_dtype))))
+
+
+def sq_linear(x: torch.Tensor, w: torch.Tensor, alpha: float, eps: float = 1e-8,
+              out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The whole path (a1..a5) on one batch. x, w and y may be CUDA tensors or
+    (pinned) host tensors; host operands are staged through the workspace."""
+    M, K = x.shape
+    N = w.shape[0]
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must have the same dtype")
+    if not (x.is_contiguous() and w.is_contiguous()):
+        raise ValueError("x and w must be contiguous")
+    dev = x.device if x.is_cuda else (w.device if w.is_cuda else torch.device("cuda", torch.cuda.current_device()))
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=dev)
+    need = sq_linear_workspace_size(M, N, K, x.dtype, y.dtype)
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    _check(_lib.sq_linear(x.data_ptr(), w.data_ptr(), _dt(x), M, N, K, float(alpha), float(eps),
+                          y.data_ptr(), _dt(y), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "sq_linear")
+    return y
+
+
+def sq_get_status(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status word."""
+    return int(_lib.sq_get_status(_stream(stream)))
+
+
+def sq_last_status_site() -> int:
+    return int(_lib.sq_last_status_site())
+
+
+def sq_last_error_string() -> str:
+    return _lib.sq_last_error_string().decode(errors="replace")
+
+
+def sq_set_wait_timeout_ms(ms: int) -> None:
+    _check(_lib.sq_set_wait_timeout_ms(int(ms)), "sq_set_wait_timeout_ms")
+
+
+def sq_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(_lib.sq_selftest_wait_timeout(int(limit_us), _stream(stream)), "sq_selftest_wait_timeout")
+
+
+def raw_status(fn_name: str, *args) -> int:
+    """Call a C entry point with raw ctypes arguments and return its status
+    (tests of the host-side argument checks)."""
+    return int(getattr(_lib, fn_name)(*args))
