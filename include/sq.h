@@ -153,6 +153,31 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* x_scale, const int8_t* wq,
                        sq_dtype out_dt, void* workspace, size_t ws_bytes,
                        sq_stream_t stream);
 
+/* ---------------------------------------------------------------- no-alloc decode GEMM
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory -- a server that has reserved the GPU's
+ * memory up front for weights and KV cache, a latency-bound decode loop that
+ * cannot afford cudaMalloc's device-wide synchronization, or a plug-in with no
+ * access to its host framework's allocator.
+ * It computes exactly what sq_w8a8_gemm computes for 1 <= M <= 16 (the split-K
+ * weight-streaming path), but keeps that path's scratch (partial sums and
+ * completion counters) in a fixed array inside the library instead of a
+ * caller workspace, and allocates nothing.
+ *   Limits: 1 <= M <= 16, M * N <= 262,144 and N <= 262,144 (1 MiB + 32 KiB of
+ *   scratch, held by every GPU that loads the library until the process
+ *   exits); larger sizes return SQ_ERR_UNSUPPORTED with a message. M == 0 or
+ *   N == 0 is a no-op.
+ *   The first call on a device looks up the scratch array's device address;
+ *   make that first call before capturing any stream into a CUDA graph.
+ *   Each call clears the part of the scratch it uses (cudaMemsetAsync on
+ *   `stream`) before its kernel. All calls on a device share the one array:
+ *   calls that overlap on the GPU (different streams, no ordering between
+ *   them) race and give wrong results; serialize them.
+ *   Other arguments, layouts and errors are those of sq_w8a8_gemm. */
+sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                               const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
+                               sq_dtype out_dt, sq_stream_t stream);
+
 /* ---------------------------------------------------------------- whole layer
  * The whole path on one batch: calibrate X and W (a1, from zero), smoothing
  * factors (a2), fold + quantize W (a3), smooth + quantize X (a4), GEMM with

@@ -4,3 +4,4 @@
 #include "sq_api.cu"
 #include "sq_quant.cu"
 #include "sq_gemm.cu"
+#include "sq_gemm_noalloc.cu"

@@ -45,6 +45,7 @@ _SIGS = {
     "sq_smooth_quant_act": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_w8a8_gemm_workspace_size": ([_i64, _i64, _i64], _sz),
     "sq_w8a8_gemm": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp], _int),
+    "sq_w8a8_gemm_noalloc": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp], _int),
     "sq_linear_workspace_size": ([_i64, _i64, _i64, _int, _int], _sz),
     "sq_linear": ([_vp, _vp, _int, _i64, _i64, _i64, _f32, _f32, _vp, _int, _vp, _sz, _vp], _int),
     "sq_get_status": ([_vp], _int),
@@ -185,6 +186,24 @@ def sq_w8a8_gemm(xq: torch.Tensor, x_scale: torch.Tensor | None, wq: torch.Tenso
                              _dev(wq, "wq"), w_scale.data_ptr() if w_scale is not None else None,
                              M, N, K, _dev(y, "y"), _dt(y), ws_ptr, ws_bytes, _stream(stream)),
            "sq_w8a8_gemm")
+    return y
+
+
+def sq_w8a8_gemm_noalloc(xq: torch.Tensor, x_scale: torch.Tensor | None, wq: torch.Tensor,
+                         w_scale: torch.Tensor | None, out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """Decode GEMM (1 <= M <= 16) for callers that cannot allocate device
+    memory: libsq keeps the scratch in a fixed array of its own. Only `y`, if
+    not given, is allocated here (by torch, for the convenience of Python
+    callers); the C call itself allocates nothing."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    _check(_lib.sq_w8a8_gemm_noalloc(_dev(xq, "xq"), x_scale.data_ptr() if x_scale is not None else None,
+                                     _dev(wq, "wq"), w_scale.data_ptr() if w_scale is not None else None,
+                                     M, N, K, _dev(y, "y"), _dt(y), _stream(stream)),
+           "sq_w8a8_gemm_noalloc")
     return y
 
 
