@@ -131,6 +131,32 @@ def test_fold_quant_weights_bitexact(dtype, rows, K):
     assert_bitexact_f32(host(wsc), osc, "w_scale")
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quant_tiny_denormal_and_extreme_rows(dtype):
+    """Rows whose maximum is below 2^-100, denormal values and quotients, and a
+    huge outlier beside tiny values: the kernels' exact fallbacks must give the
+    oracle's codes and scales."""
+    K = 1040
+    g = torch.Generator().manual_seed(12)
+    x = torch.randn(8, K, generator=g)
+    x[0] *= 1e-33
+    x[1] *= 1e-38
+    x[2] = 0.0
+    x[2, 5] = 1e-40
+    x[3, 7] = 1e30
+    x[4] *= 1e-20
+    x[5, :16] = 0.0
+    x[6] *= 1e30
+    x = x.to(dtype)
+    s = _s_for(K, 77)
+    for fn, ofn in ((sq.sq_smooth_quant_act, oracle.smooth_quant_act),
+                    (sq.sq_fold_quant_weights, oracle.fold_quant_weights)):
+        gq, gs = fn(dev(x), dev(torch.from_numpy(s)))
+        oq, osc = ofn(synth.host_array(x), s)
+        assert_equal(host(gq), oq, f"{fn.__name__} codes")
+        assert_bitexact_f32(host(gs), osc, f"{fn.__name__} scales")
+
+
 def test_quant_near_ties_and_worked_example():
     """Rows built so that many quotients sit within a few ulps of k + 1/2 and
     the 30-outlier worked example; s = 1 so x/s is exact."""

@@ -47,6 +47,8 @@ enum Site : unsigned int {
     SITE_STREAM_MMA_TMEM = 22,
     SITE_STREAM_EPILOGUE = 23,
     SITE_STREAM_DRAIN = 24,
+    SITE_QUANT_WAIT = 30,
+    SITE_QUANT_DRAIN = 31,
 };
 
 // Internal entry points used by sq_linear.

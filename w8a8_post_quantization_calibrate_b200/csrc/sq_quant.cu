@@ -48,6 +48,7 @@ struct Vec16<__nv_bfloat16> {
 };
 
 constexpr int kAbsmaxThreads = 256;
+constexpr int kAbsmaxRowsInFlight = 8;   // per warp; a block covers 64 rows per iteration
 
 template <typename T>
 __global__ void __launch_bounds__(kAbsmaxThreads)
@@ -67,18 +68,17 @@ col_absmax_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t cols,
 
     if (col < cols) {
         const uint8_t* p = x + col * (int64_t)sizeof(T);
-        int64_t r = r_begin + warp;
-        for (; r + 24 < r_end; r += 32) {
-            const uint4 v0 = ld_stream_v4(p + r * row_bytes);
-            const uint4 v1 = ld_stream_v4(p + (r + 8) * row_bytes);
-            const uint4 v2 = ld_stream_v4(p + (r + 16) * row_bytes);
-            const uint4 v3 = ld_stream_v4(p + (r + 24) * row_bytes);
-            Vec16<T>::absmax(m, v0);
-            Vec16<T>::absmax(m, v1);
-            Vec16<T>::absmax(m, v2);
-            Vec16<T>::absmax(m, v3);
+        // 8 rows per warp in flight: all loads are issued before any is used.
+        for (int64_t r = r_begin + warp; r < r_end; r += 8 * kAbsmaxRowsInFlight) {
+            uint4 v[kAbsmaxRowsInFlight];
+#pragma unroll
+            for (int u = 0; u < kAbsmaxRowsInFlight; ++u) {
+                const int64_t rr = r + 8 * u;
+                v[u] = rr < r_end ? ld_stream_v4(p + rr * row_bytes) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kAbsmaxRowsInFlight; ++u) Vec16<T>::absmax(m, v[u]);
         }
-        for (; r < r_end; r += 8) Vec16<T>::absmax(m, ld_stream_v4(p + r * row_bytes));
     }
 
     __shared__ float red[8][TILE];
@@ -216,6 +216,312 @@ row_quant_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float*
     }
 }
 
+// ============================================================== a3 / a4: fast exact path
+// The same codes and scales as row_quant_kernel (bit for bit), with the
+// per-element IEEE divisions replaced by cheaper arithmetic wherever that
+// provably cannot change a result.
+//
+// Layout. One row is handled by a group of R warps (R = 1..16, chosen from K);
+// a CTA holds several groups. Lane l of a group owns the 8-element chunks
+// l, l + 32R, ... (at most CPL of them), kept in registers between the passes.
+// Per CTA, the per-column multipliers m_j -- s_j (fold) or RN(1/s_j) (smooth,
+// __frcp_rn) -- are staged once in shared memory as fp32 (two arrays holding
+// elements 0-3 and 4-7 of every chunk, so 16-byte loads are contiguous across
+// a warp) and, for bf16 inputs, rounded to bf16 pairs.
+//
+// Row maximum. Pass 1 approximates |v_j| (v_j = RN(x_j * s_j) or
+// RN(x_j / s_j)): bf16x2 products x_j * bf16(m_j) reduced with a packed
+// absolute max (relative error < 2^-7.9), or fp32 products for fp32 inputs.
+// The group maximum m' of these bounds the exact maximum a within that error,
+// so only elements of chunks whose approximate maximum is >= m'(1 - 2^-6) can
+// attain a; their exact values (normally one chunk per row) reduced over the
+// group give a exactly.
+//
+// Codes. With r = RN(1/scale), q' = RN(RN(x * m_j) * r) differs from
+// q* = RN(v / scale) by less than 7 ulp of 127 (< 5.3e-5), so
+// round-half-even(q') = round-half-even(q*) unless q' lies within that
+// distance of a half-integer; a chunk with any q' within 2^-13 of one has
+// those codes recomputed exactly. Rounding adds 1.5*2^23: the int8 code is the
+// low byte of the sum's bits. |q'| < 127.5, so no code leaves [-127, 127].
+// Pass 2 runs on packed fp32 pairs (mul/add/sub .f32x2).
+//
+// The error bounds are relative and need normal numbers: a row whose
+// approximate maximum is below 2^-90 (this includes all-zero rows) is
+// quantized entirely with exact divisions.
+constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
+constexpr float kTieGuard = 1.0f / 8192.0f;      // >> 5.3e-5, the bound on |q' - q*|
+constexpr float kCandidate = 1.0f - 1.0f / 64.0f;
+constexpr float kSmallRow = 8.077935669463161e-28f;  // 2^-90
+constexpr int kFastMaxThreads = 512;
+constexpr int64_t kFastMaxK = 32768;             // multipliers in shared memory: 6 bytes per column
+// Chunks of 8 elements each lane keeps in registers: 8 for bf16 (32 registers), 4 for fp32.
+template <typename T> struct RowFastCPL { static constexpr int value = 8; };
+template <> struct RowFastCPL<float> { static constexpr int value = 4; };
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// Packed max of magnitudes (the sign bits of the result are not used).
+__device__ __forceinline__ uint32_t bf2_maxabs(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+template <typename T>
+struct RawChunk;
+template <>
+struct RawChunk<__nv_bfloat16> {
+    uint4 a;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { a = ld_stream_v4(p); }
+    __device__ __forceinline__ uint32_t word(int w) const { return w == 0 ? a.x : w == 1 ? a.y : w == 2 ? a.z : a.w; }
+    __device__ __forceinline__ float get(int e) const {
+        const uint32_t w = word(e >> 1);
+        return (e & 1) ? bf16_hi(w) : bf16_lo(w);
+    }
+    // elements (2p, 2p+1) as an fp32 pair
+    __device__ __forceinline__ uint64_t pair(int p) const {
+        const uint32_t w = word(p);
+        return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    // approximate max |x_e * m_e| over the chunk (bf16 arithmetic)
+    __device__ __forceinline__ float approx_max(const uint4& m16, const float (&)[8]) const {
+        const uint32_t p = bf2_maxabs(bf2_maxabs(bf2_mul(a.x, m16.x), bf2_mul(a.y, m16.y)),
+                                      bf2_maxabs(bf2_mul(a.z, m16.z), bf2_mul(a.w, m16.w)));
+        return fmaxf(fabsf(bf16_lo(p)), fabsf(bf16_hi(p)));
+    }
+};
+template <>
+struct RawChunk<float> {
+    uint4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = ld_stream_v4(p);
+        b = ld_stream_v4(p + 4);
+    }
+    __device__ __forceinline__ float get(int e) const {
+        const uint32_t w = e == 0 ? a.x : e == 1 ? a.y : e == 2 ? a.z : e == 3 ? a.w
+                         : e == 4 ? b.x : e == 5 ? b.y : e == 6 ? b.z : b.w;
+        return __uint_as_float(w);
+    }
+    __device__ __forceinline__ uint64_t pair(int p) const { return f2_pack(get(2 * p), get(2 * p + 1)); }
+    __device__ __forceinline__ float approx_max(const uint4&, const float (&mv)[8]) const {
+        float v = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v = fmaxf(v, fabsf(__fmul_rn(get(e), mv[e])));
+        return v;
+    }
+};
+
+// Exact code of one element, x the raw input: clamp(round_half_even(RN(v /
+// scale)), -127, 127) with v = RN(x * s_j) (fold) or RN(x / s_j) (smooth).
+// Out of line: these run only on the rare near-tie and small-row paths.
+template <int MODE>
+__device__ __noinline__ uint32_t exact_code(float x, float s_j, float scale) {
+    const float v = MODE == kFold ? __fmul_rn(x, s_j) : __fdiv_rn(x, s_j);
+    int qi = __float2int_rn(__fdiv_rn(v, scale));
+    qi = max(-127, min(127, qi));
+    return (uint32_t)qi & 0xffu;
+}
+
+// |v| of one element, exactly (v as above).
+template <int MODE>
+__device__ __noinline__ float exact_abs(float x, float s_j) {
+    return fabsf(MODE == kFold ? __fmul_rn(x, s_j) : __fdiv_rn(x, s_j));
+}
+
+template <int R>
+__device__ __forceinline__ float group_max(float v, float* red, int grp, int wig, int lane, int bank) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (R == 1) return v;
+    float* slot = red + (grp * 2 + bank) * R;
+    if (lane == 0) slot[wig] = v;
+    asm volatile("bar.sync %0, %1;" :: "r"(1 + grp), "r"(32 * R) : "memory");
+    v = slot[0];
+#pragma unroll
+    for (int w = 1; w < R; ++w) v = fmaxf(v, slot[w]);
+    return v;
+}
+
+template <int R>
+constexpr int row_fast_threads() { return 32 * R > 256 ? 32 * R : 256; }
+
+template <typename T, int MODE, int R, int CPL>
+__global__ void __launch_bounds__(row_fast_threads<R>(), R >= 16 ? 1 : 3)
+row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
+                      int8_t* __restrict__ q, float* __restrict__ scale_out) {
+    extern __shared__ float smem[];
+    const int64_t nchunks = K >> 3;
+    float* mul_lo = smem;                                                // [nchunks][4] fp32, elements 0..3
+    float* mul_hi = smem + nchunks * 4;                                  // [nchunks][4] fp32, elements 4..7
+    uint32_t* mul16 = reinterpret_cast<uint32_t*>(smem + nchunks * 8);   // [nchunks][4] bf16 pairs
+    float* red = smem + nchunks * 12;                                    // [groups][2][R]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int groups = blockDim.x / (32 * R);
+    const int grp = warp / R, wig = warp % R;
+    const int gl = wig * 32 + lane;          // lane index inside the group
+
+    for (int64_t c = threadIdx.x; c < nchunks; c += blockDim.x) {
+        float4 a = __ldg(reinterpret_cast<const float4*>(s + c * 8));
+        float4 b = __ldg(reinterpret_cast<const float4*>(s + c * 8 + 4));
+        if (MODE == kSmooth) {
+            a = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
+            b = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
+        }
+        *reinterpret_cast<float4*>(mul_lo + c * 4) = a;
+        *reinterpret_cast<float4*>(mul_hi + c * 4) = b;
+        *reinterpret_cast<uint4*>(mul16 + c * 4) =
+            make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+    }
+    __syncthreads();
+
+    const uint64_t mag2 = f2_pack(kMagic, kMagic);
+    int bank = 0;
+    for (int64_t row = (int64_t)blockIdx.x * groups + grp; row < rows; row += (int64_t)gridDim.x * groups) {
+        const T* rin = in + row * K;
+        RawChunk<T> raw[CPL];
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int64_t c = gl + (int64_t)i * 32 * R;
+            if (c < nchunks) raw[i].load(rin + c * 8);
+        }
+
+        // ---- pass 1: approximate chunk maxima
+        float cm[CPL];
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int64_t c = gl + (int64_t)i * 32 * R;
+            cm[i] = 0.0f;
+            if (c < nchunks) {
+                float mv[8];
+                if (sizeof(T) == 4) {
+                    const float4 a = *reinterpret_cast<const float4*>(mul_lo + c * 4);
+                    const float4 b = *reinterpret_cast<const float4*>(mul_hi + c * 4);
+                    mv[0] = a.x; mv[1] = a.y; mv[2] = a.z; mv[3] = a.w;
+                    mv[4] = b.x; mv[5] = b.y; mv[6] = b.z; mv[7] = b.w;
+                }
+                const uint4 m16 = sizeof(T) == 2 ? *reinterpret_cast<const uint4*>(mul16 + c * 4) : make_uint4(0u, 0u, 0u, 0u);
+                cm[i] = raw[i].approx_max(m16, mv);
+                m = fmaxf(m, cm[i]);
+            }
+        }
+        const float mrow = group_max<R>(m, red, grp, wig, lane, bank);
+        bank ^= 1;
+        int8_t* rq = q + row * K;
+
+        if (!(mrow >= kSmallRow)) {
+            // zero, tiny or near-underflow row: exact maximum and codes
+            float ex = 0.0f;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int64_t c = gl + (int64_t)i * 32 * R;
+                if (c < nchunks)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(raw[i].get(e), __ldg(s + c * 8 + e)));
+            }
+            const float a = group_max<R>(ex, red, grp, wig, lane, bank);
+            bank ^= 1;
+            const float scale = a == 0.0f ? 1.0f : __fdiv_rn(a, 127.0f);
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int64_t c = gl + (int64_t)i * 32 * R;
+                if (c < nchunks) {
+                    uint32_t b[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        b[e] = a == 0.0f ? 0u : exact_code<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), scale);
+                    *reinterpret_cast<uint2*>(rq + c * 8) =
+                        make_uint2(b[0] | b[1] << 8 | b[2] << 16 | b[3] << 24, b[4] | b[5] << 8 | b[6] << 16 | b[7] << 24);
+                }
+            }
+            if (gl == 0) scale_out[row] = scale;
+            continue;
+        }
+
+        // exact values of the candidates (normally one chunk per row)
+        const float tau = __fmul_rn(mrow, kCandidate);
+        float ex = 0.0f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            if (cm[i] >= tau) {
+                const int64_t c = gl + (int64_t)i * 32 * R;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(raw[i].get(e), __ldg(s + c * 8 + e)));
+            }
+        }
+        const float amax = group_max<R>(ex, red, grp, wig, lane, bank);
+        bank ^= 1;
+
+        // ---- pass 2: codes
+        const float scale = __fdiv_rn(amax, 127.0f);
+        const float r = __frcp_rn(scale);
+        const uint64_t r2 = f2_pack(r, r);
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int64_t c = gl + (int64_t)i * 32 * R;
+            if (c < nchunks) {
+                const float4 a = *reinterpret_cast<const float4*>(mul_lo + c * 4);
+                const float4 b = *reinterpret_cast<const float4*>(mul_hi + c * 4);
+                const uint64_t mp[4] = {f2_pack(a.x, a.y), f2_pack(a.z, a.w), f2_pack(b.x, b.y), f2_pack(b.z, b.w)};
+                uint32_t t[8];
+                bool near_tie = false;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const uint64_t q2 = f2_mul(f2_mul(raw[i].pair(p), mp[p]), r2);
+                    const uint64_t t2 = f2_add(q2, mag2);
+                    const uint64_t d2 = f2_sub(q2, f2_sub(t2, mag2));
+                    float t0, t1, d0, d1;
+                    f2_unpack(t2, t0, t1);
+                    f2_unpack(d2, d0, d1);
+                    t[2 * p] = __float_as_uint(t0);
+                    t[2 * p + 1] = __float_as_uint(t1);
+                    near_tie |= fabsf(d0) >= 0.5f - kTieGuard;
+                    near_tie |= fabsf(d1) >= 0.5f - kTieGuard;
+                }
+                if (near_tie) {
+                    const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float qv = __fmul_rn(__fmul_rn(raw[i].get(e), mv[e]), r);
+                        const float d = __fsub_rn(qv, __fsub_rn(__fadd_rn(qv, kMagic), kMagic));
+                        if (fabsf(d) >= 0.5f - kTieGuard) t[e] = exact_code<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), scale);
+                    }
+                }
+                const uint32_t lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+                const uint32_t hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+                *reinterpret_cast<uint2*>(rq + c * 8) = make_uint2(lo, hi);
+            }
+        }
+        if (gl == 0) scale_out[row] = scale;
+    }
+}
+
 // ============================================================== host side
 namespace {
 
@@ -248,10 +554,53 @@ int pow2ceil(int64_t v) {
     return p;
 }
 
+template <typename T, int MODE, int R>
+sq_status launch_row_quant_fast_inst(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
+                                     float* scale, cudaStream_t st) {
+    constexpr int CPL = RowFastCPL<T>::value;
+    static bool attr_done[64] = {};
+    const DeviceInfo& di = device_info();
+    const int threads = 32 * R > 256 ? 32 * R : 256;
+    const int groups = threads / (32 * R);
+    const size_t smem = (size_t)K * 6 + (size_t)groups * 2 * R * sizeof(float);
+    auto kern = row_quant_fast_kernel<T, MODE, R, CPL>;
+    if (!attr_done[di.device & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(kFastMaxK * 6 + 1024));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row_quant_fast_kernel)");
+        attr_done[di.device & 63] = true;
+    }
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (per_sm < 1) per_sm = 1;
+    const int64_t need = (rows + groups - 1) / groups;
+    const int64_t max_blocks = (int64_t)di.sm_count * per_sm;
+    const int grid = (int)(need < max_blocks ? need : max_blocks);
+    kern<<<grid, threads, smem, st>>>(static_cast<const T*>(in), rows, K, s, q, scale);
+    return check_launch("row_quant_fast_kernel");
+}
+
 template <typename T, int MODE>
 sq_status launch_row_quant(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
                            float* scale, cudaStream_t st) {
+    constexpr int CPL = RowFastCPL<T>::value;
     const int64_t nchunks = K / 8;
+    // the fewest warps per row whose lanes hold the row in CPL chunks each
+    if (K <= kFastMaxK) {
+        for (int R = 1; R <= 16; R *= 2) {
+            if (nchunks <= (int64_t)32 * R * CPL) {
+                switch (R) {
+                    case 1: return launch_row_quant_fast_inst<T, MODE, 1>(in, rows, K, s, q, scale, st);
+                    case 2: return launch_row_quant_fast_inst<T, MODE, 2>(in, rows, K, s, q, scale, st);
+                    case 4: return launch_row_quant_fast_inst<T, MODE, 4>(in, rows, K, s, q, scale, st);
+                    case 8: return launch_row_quant_fast_inst<T, MODE, 8>(in, rows, K, s, q, scale, st);
+                    default: return launch_row_quant_fast_inst<T, MODE, 16>(in, rows, K, s, q, scale, st);
+                }
+            }
+        }
+    }
+    // longer rows: the IEEE-division kernel
     int64_t tpb = pow2ceil((nchunks + 3) / 4);
     if (tpb < 128) tpb = 128;
     if (tpb > 1024) tpb = 1024;
@@ -309,17 +658,21 @@ sq_status calibrate_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_
     const int es = dt == SQ_F32 ? 4 : 2;
     const int64_t tile = 32 * (16 / es);
     const int64_t ct = (cols + tile - 1) / tile;
-    const int64_t bytes = rows * cols * es;
-    int64_t target = bytes / 65536;
-    const int64_t cap = (int64_t)device_info().sm_count * 16;
-    if (target > cap) target = cap;
+    // About one wave of 256-thread blocks (8 per SM); every block covers a
+    // multiple of the 64 rows it reads per iteration.
+    const int64_t step_rows = 8 * kAbsmaxRowsInFlight;
+    const int64_t target = (int64_t)device_info().sm_count * 8;
     int64_t rc = target / ct;
     if (rc < 1) rc = 1;
-    const int64_t rc_max = (rows + 7) / 8;
-    if (rc > rc_max) rc = rc_max;
-    if (rc > 65535) rc = 65535;
-    const int64_t per = (rows + rc - 1) / rc;
+    int64_t per = (rows + rc - 1) / rc;
+    per = (per + step_rows - 1) / step_rows * step_rows;
     rc = (rows + per - 1) / per;
+    if (rc > 65535) {
+        rc = 65535;
+        per = (rows + rc - 1) / rc;
+        per = (per + step_rows - 1) / step_rows * step_rows;
+        rc = (rows + per - 1) / per;
+    }
     if (ct > 2147483647LL) { set_error("cols too large"); return SQ_ERR_UNSUPPORTED; }
     dim3 grid((unsigned)ct, (unsigned)rc);
     if (dt == SQ_F32)
