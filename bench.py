@@ -302,7 +302,7 @@ def run_ours(args, world, rank, local):
         kernels[n] = entry
     gemm_ms = per_kernel["a5_w8a8_gemm"]
     achieved = ops / (gemm_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "gemm_tiled_kernel (a5)", "achieved": round(achieved, 1),
+    roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel (a5, paired-SM tcgen05)", "achieved": round(achieved, 1),
                 "peak": round(int8_peak, 1), "unit": "TOPS", "frac": round(achieved / int8_peak, 4),
                 "traffic": load_traffic(),
                 "peak_source": f"{peak_src}: bf16 {bf16_peak} TFLOP/s (burst) x {INT8_OVER_BF16} nominal "

@@ -300,6 +300,255 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
 }
 
+// ================================================================== prefill, paired SMs
+// A cluster of two CTAs on a pair of SMs computes 256 x 256 output tiles with
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=32), issued by CTA 0. Each CTA
+// loads only its own halves -- 128 rows of A (its rows of the tile) and 128
+// rows of B (half of the tile's columns) -- into a 6-stage ring; the MMA reads
+// the B half of the other CTA directly. Both CTAs' loads signal CTA 0's "full"
+// barrier (one arrival, 64 KB of transactions); CTA 0's commits arrive on the
+// "empty" and "accumulator full" barriers of both CTAs (commit multicast, a
+// barrier arrival -- no data multicast). Each CTA's TMEM holds its 128 rows x
+// 256 columns of the accumulator (double-buffered); its epilogue warps drain
+// it and arrive on CTA 0's "accumulator empty" barrier.
+constexpr int P_STAGES = 6;
+constexpr uint32_t P_A_STAGE = 128 * BK;        // 16 KB: this CTA's 128 rows of A
+constexpr uint32_t P_B_STAGE = 128 * BK;        // 16 KB: this CTA's 128 rows of B
+constexpr uint32_t P_TX_BYTES = 2 * (P_A_STAGE + P_B_STAGE);   // both CTAs, per stage
+constexpr uint32_t IDESC_PAIR = make_idesc_i8(256, 256);
+
+constexpr size_t pair_smem_bytes() {
+    return 1024 + P_STAGES * (P_A_STAGE + P_B_STAGE) + 256;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cta0, int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        :: "r"(dst), "l"(tmap), "r"(bar_cta0), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Arrive once on `bar` in both CTAs of the pair when the MMAs issued so far are done.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 :: "r"(bar), "h"((uint16_t)3) : "memory");
+}
+// shared::cluster address of the same shared-memory offset in CTA 0 of the cluster.
+__device__ __forceinline__ uint32_t cta0_addr(uint32_t local_addr) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(r) : "r"(local_addr));
+    return r;
+}
+// Arrive once on `bar` of CTA 0 only when the MMAs issued so far are done.
+__device__ __forceinline__ void mma_commit_cta0(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 :: "r"(bar), "h"((uint16_t)1) : "memory");
+}
+__device__ __forceinline__ void arrive_on_cta0(uint32_t local_bar) {
+    asm volatile("{\n\t.reg .b32 ra;\n\t"
+                 "mapa.shared::cluster.u32 ra, %0, 0;\n\t"
+                 "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+                 :: "r"(local_bar) : "memory");
+}
+template <int NCOLS>
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t holder_smem) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(holder_smem), "n"(NCOLS) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+template <int NCOLS>
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "n"(NCOLS) : "memory");
+}
+
+template <int OUT>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const float* __restrict__ x_scale, const float* __restrict__ w_scale,
+                 void* __restrict__ y, int M, int N, int K, long long wait_limit) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + P_STAGES * P_A_STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + P_STAGES * P_B_STAGE);
+    // bars: full[P_STAGES] | empty[P_STAGES] | tfull[2] | tempty[2] | drain
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * P_STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    __shared__ int no_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int num_m = (M + 255) / 256, num_n = (N + 255) / 256;
+    const int num_tiles = num_m * num_n;
+    const int num_kb = (K + BK - 1) / BK;
+
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+    const int FULL = 0, EMPTY = P_STAGES, TFULL = 2 * P_STAGES, TEMPTY = 2 * P_STAGES + 2, DRAIN = 2 * P_STAGES + 4;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(bar(FULL + s), 1);
+            mbar_init(bar(EMPTY + s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar(TFULL + a), 1);
+            mbar_init(bar(TEMPTY + a), 8);   // 4 epilogue warps in each CTA
+        }
+        mbar_init(bar(DRAIN), 1);
+        *abort_flag = 0;
+        no_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair<TMEM_COLS>(smem_u32(tmem_holder));
+        tc_fence_before();
+    }
+    // barriers of both CTAs initialised before either uses the other's
+    __syncwarp();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+                int mb, nb;
+                tile_coords(tile, num_m, num_n, mb, nb);
+                const int arow = mb * 256 + (int)rank * 128;
+                const int brow = nb * 256 + (int)rank * 128;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar(EMPTY + stage), phase ^ 1, wait_limit, abort_flag, SITE_GEMM_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full0 = cta0_addr(bar(FULL + stage));
+                    if (rank == 0) mbar_arrive_expect_tx(bar(FULL + stage), P_TX_BYTES);
+                    tma_load_2d_pair(smem_u32(sA + stage * P_A_STAGE), &tmA, full0, kb * BK, arow);
+                    tma_load_2d_pair(smem_u32(sB + stage * P_B_STAGE), &tmB, full0, kb * BK, brow);
+                    ++issued;
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok || *abort_flag) {
+                // Copies in flight must land before the pair exits. CTA 0 can see
+                // its full barriers complete; both CTAs also wait a bounded grace time.
+                if (rank == 0) {
+                    for (int s = 0; s < P_STAGES; ++s) {
+                        const long long cnt = issued / P_STAGES + (s < issued % P_STAGES ? 1 : 0);
+                        if (cnt > 0)
+                            mbar_wait(bar(FULL + s), (uint32_t)((cnt - 1) & 1), wait_limit, &no_abort, SITE_GEMM_DRAIN);
+                    }
+                }
+                const long long t0 = clock64();
+                while (clock64() - t0 < 2000000) { }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer (CTA 0)
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+                if (!mbar_wait(bar(TEMPTY + acc), acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM_MMA_TMEM)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(bar(FULL + stage), phase, wait_limit, abort_flag, SITE_GEMM_MMA_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * P_A_STAGE);
+                    const uint32_t b0 = smem_u32(sB + stage * P_B_STAGE);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k)
+                        mma_i8_pair(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
+                                    make_sw128_kmajor_desc(b0 + k * UMMA_K), IDESC_PAIR, (kb | k) != 0 ? 1u : 0u);
+                    mma_commit_pair(bar(EMPTY + stage));
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit_pair(bar(TFULL + acc));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            mma_commit_cta0(bar(DRAIN));
+            mbar_wait(bar(DRAIN), 0, wait_limit, &no_abort, SITE_GEMM_DRAIN);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (warps 2..5, both CTAs)
+        const int quarter = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < num_tiles; tile += npairs) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            if (!mbar_wait(bar(TFULL + acc), acc_phase, wait_limit, abort_flag, SITE_GEMM_EPILOGUE)) break;
+            tc_fence_after();
+            const int64_t row = (int64_t)mb * 256 + rank * 128 + quarter * 32 + lane;
+            const bool row_ok = row < M;
+            const float sa = (OUT != kOutI32 && row_ok) ? __ldg(x_scale + row) : 0.0f;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; c += 2) {
+                uint32_t r0[32], r1[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, r0);
+                tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
+                tmem_wait_ld();
+                const int col0 = nb * BN + c * 32;
+                if (row_ok && col0 < N) store_row32<OUT>(y, row, col0, N, r0, sa, w_scale);
+                if (row_ok && col0 + 32 < N) store_row32<OUT>(y, row, col0 + 32, N, r1, sa, w_scale);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(bar(TEMPTY + acc));
+                else arrive_on_cta0(bar(TEMPTY + acc));
+            }
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+
+    // neither CTA leaves while the other may still touch its shared memory or TMEM
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair<TMEM_COLS>(tmem_base);
+    }
+}
+
 // ================================================================== decode
 // Work unit = (row tile of W, k-block). CTA c owns units [c*U/G, (c+1)*U/G);
 // a maximal run of its units inside one row tile is a segment, accumulated in
@@ -564,6 +813,34 @@ sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float
 }
 
 template <int OUT>
+sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
+                      int M, int N, int K, cudaStream_t st) {
+    static bool attr_done[64] = {};
+    const DeviceInfo& di = device_info();
+    const size_t smem = pair_smem_bytes();
+    sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT>, smem, attr_done[di.device & 63]);
+    if (r != SQ_OK) return r;
+    const int tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int max_pairs = di.sm_count / 2;
+    const int pairs = tiles < max_pairs ? tiles : max_pairs;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<OUT>, ta, tb, xs, wsc, y, M, N, K, wait_limit_cycles());
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(gemm_pair_kernel)");
+    return check_launch("gemm_pair_kernel");
+}
+
+template <int OUT>
 sq_status launch_stream(const CUtensorMap& tw, const CUtensorMap& tx, const float* xs, const float* wsc, void* y,
                         int M, int N, int K, int32_t* ws_acc, unsigned int* counts, cudaStream_t st) {
     static bool attr_done[64] = {};
@@ -636,6 +913,16 @@ sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq
         }
     }
     CUtensorMap ta, tb;
+    if (M > 128) {
+        // paired SMs: each CTA loads 128-row boxes of A and of B
+        if ((r = make_map_i8(&ta, xq, M, K, 128)) != SQ_OK) return r;
+        if ((r = make_map_i8(&tb, wq, N, K, 128)) != SQ_OK) return r;
+        switch (out) {
+            case kOutF32: return launch_pair<kOutF32>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
+            case kOutBF16: return launch_pair<kOutBF16>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
+            default: return launch_pair<kOutI32>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
+        }
+    }
     if ((r = make_map_i8(&ta, xq, M, K, BM)) != SQ_OK) return r;
     if ((r = make_map_i8(&tb, wq, N, K, BN)) != SQ_OK) return r;
     switch (out) {
