@@ -201,17 +201,28 @@ def kernel_bytes(M, N, K, in_es, out_es):
     }
 
 
+def workload_inputs(name: str, decode_m: int):
+    """(workload, x, w, alpha, out bytes) for a workload name; mlp_decode_7b
+    takes its token count from --decode-m and uses the gate projection."""
+    wl = synth.WORKLOADS[name]
+    if name == "mlp_decode_7b":
+        x, w = synth.make_decode(decode_m, "gate")
+    else:
+        x, w = synth.make(name)
+    return wl, x, w
+
+
 def run_ours(args, world, rank, local):
     from w8a8_post_quantization_calibrate_b200 import sq
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     init_dist(world, "nccl")
-    wl = synth.WORKLOADS[WORKLOAD]
-    M, N, K = wl.T, wl.N, wl.K
-    x_cpu, w_cpu = synth.make(WORKLOAD)
+    wl, x_cpu, w_cpu = workload_inputs(args.workload, args.decode_m)
+    M, K = x_cpu.shape
+    N = w_cpu.shape[0]
     x = x_cpu.to(dev)
     w = w_cpu.to(dev)
-    in_es, out_es = 2, 2
+    in_es, out_es = x_cpu.element_size(), torch.empty(0, dtype=wl.out_dtype).element_size()
     stream = torch.cuda.current_stream(dev)
 
     xmax = torch.zeros(K, dtype=torch.float32, device=dev)
@@ -223,7 +234,7 @@ def run_ours(args, world, rank, local):
     wsc = torch.empty(N, dtype=torch.float32, device=dev)
     xq = torch.empty((M, K), dtype=torch.int8, device=dev)
     xsc = torch.empty(M, dtype=torch.float32, device=dev)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((M, N), dtype=wl.out_dtype, device=dev)
     gws = sq.gemm_workspace(M, N, K, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -302,29 +313,38 @@ def run_ours(args, world, rank, local):
         kernels[n] = entry
     gemm_ms = per_kernel["a5_w8a8_gemm"]
     achieved = ops / (gemm_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel (a5, paired-SM tcgen05)", "achieved": round(achieved, 1),
-                "peak": round(int8_peak, 1), "unit": "TOPS", "frac": round(achieved / int8_peak, 4),
-                "traffic": load_traffic(),
-                "peak_source": f"{peak_src}: bf16 {bf16_peak} TFLOP/s (burst) x {INT8_OVER_BF16} nominal "
-                               f"int8/bf16 ratio",
-                "algorithmic_ops_per_launch": ops}
+    if M > 16:
+        roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel (a5, paired-SM tcgen05)" if M > 128
+                    else "gemm_tiled_kernel (a5)",
+                    "achieved": round(achieved, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
+                    "frac": round(achieved / int8_peak, 4), "traffic": load_traffic() if M > 128 else None,
+                    "peak_source": f"{peak_src}: bf16 {bf16_peak} TFLOP/s (burst) x {INT8_OVER_BF16} nominal "
+                                   f"int8/bf16 ratio",
+                    "algorithmic_ops_per_launch": ops}
+    else:
+        gbs = kb["a5_w8a8_gemm"] / (gemm_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "gemm_stream_kernel (a5, split-K weight streaming)",
+                    "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                    "traffic": None, "peak_source": f"{peak_src}: hbm_gbs",
+                    "algorithmic_bytes_per_launch": kb["a5_w8a8_gemm"]}
 
     # end to end through the public API: pinned host X and W in, host Y out
     e2e = None
     if args.e2e_steps > 0:
         xh = x_cpu.pin_memory()
         wh = w_cpu.pin_memory()
-        yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-        lws = torch.zeros(sq.sq_linear_workspace_size(M, N, K), dtype=torch.uint8, device=dev)
+        yh = torch.empty((M, N), dtype=wl.out_dtype).pin_memory()
+        lws = torch.zeros(sq.sq_linear_workspace_size(M, N, K, x_cpu.dtype, wl.out_dtype), dtype=torch.uint8,
+                          device=dev)
         for _ in range(2):
-            sq.sq_linear(xh, wh, wl.alpha, y=yh, workspace=lws, stream=stream)
+            sq.sq_linear(xh, wh, wl.alpha, out_dtype=wl.out_dtype, y=yh, workspace=lws, stream=stream)
         torch.cuda.synchronize(dev)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.e2e_steps)]
         barrier(world)
         for a, b in ev:
             a.record(stream)
-            sq.sq_linear(xh, wh, wl.alpha, y=yh, workspace=lws, stream=stream)
+            sq.sq_linear(xh, wh, wl.alpha, out_dtype=wl.out_dtype, y=yh, workspace=lws, stream=stream)
             b.record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
@@ -350,7 +370,9 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded outlier-bearing activations, N(0,1/64) weights)",
-        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "in_dtype": "bf16", "out_dtype": "bf16",
+        "config": {"workload": args.workload, "M": M, "N": N, "K": K,
+                   "in_dtype": str(x_cpu.dtype).replace("torch.", ""),
+                   "out_dtype": str(wl.out_dtype).replace("torch.", ""),
                    "alpha": wl.alpha, "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "step": "a1(X) a1(W) a2 a3 a4 a5, one stream"},
@@ -366,11 +388,12 @@ def run_reference(args, world, rank):
     reference arm: each step is one bounded sample of the workload."""
     if rank != 0:
         return None
-    wl = synth.WORKLOADS[WORKLOAD]
-    x_cpu, w_cpu = synth.make(WORKLOAD)
+    wl, x_cpu, w_cpu = workload_inputs(args.workload, args.decode_m)
+    M, K = x_cpu.shape
+    N = w_cpu.shape[0]
     budget = max(0.002, args.reference_budget_s / max(1, args.steps + args.warmup))
     # size the slice so one step stays within the budget
-    tokens, rows = 64, 256
+    tokens, rows = min(64, M), min(256, N)
     _, _, _, per = oracle_sample(x_cpu, w_cpu, wl.alpha, 0.0, tokens, rows)
     while per > budget and tokens > 1:
         tokens //= 2
@@ -381,17 +404,18 @@ def run_reference(args, world, rank):
     for _ in range(args.steps):
         oracle_sample(x_cpu, w_cpu, wl.alpha, 0.0, tokens, rows)
     el = time.perf_counter() - t0
-    ops = 2.0 * tokens * rows * wl.K
+    ops = 2.0 * tokens * rows * K
     value = ops * args.steps / el / 1e12
     import oracle
     desc = (f"oracle whole path (a1..a5) on a {tokens}-token x {rows}-output-channel slice of the "
-            f"workload per step (K={wl.K}); value = int8 ops of the slice / time")
+            f"workload per step (K={K}); value = int8 ops of the slice / time")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic", "config": {"workload": WORKLOAD, "M": wl.T, "N": wl.N, "K": wl.K,
-                                        "in_dtype": "bf16", "out_dtype": "bf16", "alpha": wl.alpha},
+        "data": "synthetic", "config": {"workload": args.workload, "M": M, "N": N, "K": K,
+                                        "in_dtype": str(x_cpu.dtype).replace("torch.", ""),
+                                        "out_dtype": str(wl.out_dtype).replace("torch.", ""), "alpha": wl.alpha},
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -404,6 +428,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=WORKLOAD,
+                    help="the measured configuration is the 7B QKV prefill; the others are for profiling")
+    ap.add_argument("--decode-m", type=int, default=16, choices=synth.DECODE_MS)
     ap.add_argument("--e2e-steps", type=int, default=10, help="steps of the end-to-end measurement")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)

@@ -372,7 +372,7 @@ template <int R>
 constexpr int row_fast_threads() { return 32 * R > 256 ? 32 * R : 256; }
 
 template <typename T, int MODE, int R, int CPL>
-__global__ void __launch_bounds__(row_fast_threads<R>(), R >= 16 ? 1 : 3)
+__global__ void __launch_bounds__(row_fast_threads<R>(), R >= 16 ? 1 : (R >= 8 ? 2 : 4))
 row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
                       int8_t* __restrict__ q, float* __restrict__ scale_out) {
     extern __shared__ float smem[];
@@ -402,13 +402,40 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
 
     const uint64_t mag2 = f2_pack(kMagic, kMagic);
     int bank = 0;
-    for (int64_t row = (int64_t)blockIdx.x * groups + grp; row < rows; row += (int64_t)gridDim.x * groups) {
+    // Long rows (R >= 8) double-buffer the row in registers: the next row's
+    // loads are issued before the current row is processed.
+    constexpr bool kPrefetch = R >= 8;
+    const int64_t stride = (int64_t)gridDim.x * groups;
+    RawChunk<T> nxt[CPL];
+    if (kPrefetch) {
+        const int64_t row = (int64_t)blockIdx.x * groups + grp;
+        if (row < rows) {
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int64_t c = gl + (int64_t)i * 32 * R;
+                if (c < nchunks) nxt[i].load(in + row * K + c * 8);
+            }
+        }
+    }
+    for (int64_t row = (int64_t)blockIdx.x * groups + grp; row < rows; row += stride) {
         const T* rin = in + row * K;
         RawChunk<T> raw[CPL];
+        if (kPrefetch) {
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int64_t c = gl + (int64_t)i * 32 * R;
-            if (c < nchunks) raw[i].load(rin + c * 8);
+            for (int i = 0; i < CPL; ++i) raw[i] = nxt[i];
+            if (row + stride < rows) {
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) {
+                    const int64_t c = gl + (int64_t)i * 32 * R;
+                    if (c < nchunks) nxt[i].load(in + (row + stride) * K + c * 8);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int64_t c = gl + (int64_t)i * 32 * R;
+                if (c < nchunks) raw[i].load(rin + c * 8);
+            }
         }
 
         // ---- pass 1: approximate chunk maxima
