@@ -717,18 +717,27 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                 // sums are in ws_acc. Write Y and leave the workspace zeroed.
                 __threadfence();
                 if (n < N) {
+                    // all partial sums (and scales) are loaded before any is used
                     const float sw = (OUT != kOutI32) ? __ldg(w_scale + n) : 0.0f;
-                    for (int t = 0; t < M; ++t) {
-                        int32_t* p = ws_acc + (int64_t)t * N + n;
-                        const int32_t a = __ldcg(p);
-                        *p = 0;
-                        const int64_t o = (int64_t)t * N + n;
-                        if (OUT == kOutI32) {
-                            static_cast<int32_t*>(y)[o] = a;
-                        } else {
-                            const float v = dequant(a, __ldg(x_scale + t), sw);
-                            if (OUT == kOutF32) static_cast<float*>(y)[o] = v;
-                            else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+                    int32_t a[S_BN];
+                    float sa[S_BN];
+#pragma unroll
+                    for (int t = 0; t < S_BN; ++t) {
+                        a[t] = t < M ? __ldcg(ws_acc + (int64_t)t * N + n) : 0;
+                        sa[t] = (OUT != kOutI32 && t < M) ? __ldg(x_scale + t) : 0.0f;
+                    }
+#pragma unroll
+                    for (int t = 0; t < S_BN; ++t) {
+                        if (t < M) {
+                            const int64_t o = (int64_t)t * N + n;
+                            ws_acc[o] = 0;
+                            if (OUT == kOutI32) {
+                                static_cast<int32_t*>(y)[o] = a[t];
+                            } else {
+                                const float v = dequant(a[t], sa[t], sw);
+                                if (OUT == kOutF32) static_cast<float*>(y)[o] = v;
+                                else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+                            }
                         }
                     }
                 }
