@@ -40,6 +40,12 @@ MUTATIONS = {
     "fold_divides": 10,
     "colmax_no_abs": 11,
     "smooth_wrong_index": 12,
+    "tensor_max_unsmoothed": 13,
+    "norm_no_eps": 14,
+    "norm_mean_abs": 15,
+    "split_max_all": 16,
+    "split_drop_outliers": 17,
+    "e4m3_truncate": 18,
 }
 
 _lock = threading.Lock()
@@ -87,6 +93,22 @@ def lib():
             L.sqo_w8a8_f64.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
             L.sqo_rel_frobenius_f64.argtypes = [vp, vp, i64]
             L.sqo_rel_frobenius_f64.restype = f64
+            L.sqo_tensor_absmax.argtypes = [vp, ctypes.c_int, i64, i64, vp, vp]
+            L.sqo_quant_act_per_tensor.argtypes = [vp, ctypes.c_int, i64, i64, vp, f32, vp, vp]
+            L.sqo_fold_norm_gain.argtypes = [vp, ctypes.c_int, i64, vp, vp]
+            L.sqo_rmsnorm_quant_act.argtypes = [vp, ctypes.c_int, i64, i64, vp, f32, vp, vp, vp, vp]
+            L.sqo_outlier_split.argtypes = [vp, i64, f32, vp, vp]
+            L.sqo_outlier_split.restype = i64
+            L.sqo_quant_bulk.argtypes = [vp, ctypes.c_int, i64, i64, vp, vp, vp]
+            L.sqo_gather_columns.argtypes = [vp, ctypes.c_int, i64, i64, vp, i64, i64, vp]
+            L.sqo_dequant_split.argtypes = [vp, vp, vp, i64, i64, vp, vp, i64, i64, vp, vp, vp]
+            L.sqo_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+            L.sqo_e4m3_to_f64.restype = f64
+            L.sqo_e4m3_from_f64.argtypes = [f64]
+            L.sqo_e4m3_from_f64.restype = ctypes.c_uint8
+            L.sqo_quant_row_e4m3.argtypes = [vp, i64, vp, vp]
+            L.sqo_quant_rows_e4m3_f64.argtypes = [vp, i64, i64, vp, vp]
+            L.sqo_w8a8_e4m3_f64.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
             L.sqo_num_threads.restype = ctypes.c_int
             L.sqo_set_num_threads.argtypes = [ctypes.c_int]
             _lib = L
@@ -294,3 +316,186 @@ def w8a8_error_f64(X: np.ndarray, W: np.ndarray, Y: np.ndarray | None = None) ->
     if Y is None:
         Y = matmul_xwT_f64(X, W)
     return rel_frobenius_f64(w8a8_f64(X, W), Y)
+
+
+# ---------------------------------------------------------------- next steps
+def _opt(a):
+    return None if a is None else _p(a)
+
+
+def tensor_absmax(x: np.ndarray, s: np.ndarray | None, amax: float = 0.0) -> np.float32:
+    """Running max of |RN(x / s_j)| over a whole batch (s None: of |x|)."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    s = None if s is None else np.ascontiguousarray(s, dtype=np.float32)
+    out = np.array([amax], np.float32)
+    lib().sqo_tensor_absmax(_p(x), _dt(x), rows, cols, _opt(s), _p(out))
+    return out[0]
+
+
+def quant_act_per_tensor(x: np.ndarray, s: np.ndarray | None, amax: float):
+    """Per-tensor int8 of RN(x / s) with range amax -> (codes [T,K], x_scale [T])."""
+    x = np.ascontiguousarray(x)
+    T, K = x.shape
+    s = None if s is None else np.ascontiguousarray(s, dtype=np.float32)
+    xq = np.empty((T, K), np.int8)
+    xs = np.empty(T, np.float32)
+    lib().sqo_quant_act_per_tensor(_p(x), _dt(x), T, K, _opt(s), float(np.float32(amax)), _p(xq), _p(xs))
+    return xq, xs
+
+
+def fold_norm_gain(g: np.ndarray, s: np.ndarray) -> np.ndarray:
+    g = np.ascontiguousarray(g)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    gf = np.empty(s.shape[0], np.float32)
+    lib().sqo_fold_norm_gain(_p(g), _dt(g), s.shape[0], _p(s), _p(gf))
+    return gf
+
+
+def rmsnorm_quant_act(x: np.ndarray, gf: np.ndarray, eps: float, r_in: np.ndarray | None = None):
+    """RMSNorm(x; gain gf) then per-token int8 -> (codes, x_scale, r)."""
+    x = np.ascontiguousarray(x)
+    T, K = x.shape
+    gf = np.ascontiguousarray(gf, dtype=np.float32)
+    r_in = None if r_in is None else np.ascontiguousarray(r_in, dtype=np.float32)
+    xq = np.empty((T, K), np.int8)
+    xs = np.empty(T, np.float32)
+    r = np.empty(T, np.float32)
+    lib().sqo_rmsnorm_quant_act(_p(x), _dt(x), T, K, _p(gf), float(eps), _opt(r_in), _p(xq), _p(xs), _p(r))
+    return xq, xs, r
+
+
+def outlier_split(xmax: np.ndarray, threshold: float):
+    """-> (keep float32 [K] of 1/0, outlier indices int32 ascending)."""
+    xmax = np.ascontiguousarray(xmax, dtype=np.float32)
+    K = xmax.shape[0]
+    keep = np.empty(K, np.float32)
+    idx = np.empty(K, np.int32)
+    n = lib().sqo_outlier_split(_p(xmax), K, float(threshold), _p(keep), _p(idx))
+    return keep, idx[:n].copy()
+
+
+def quant_bulk(x: np.ndarray, keep: np.ndarray):
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    keep = np.ascontiguousarray(keep, dtype=np.float32)
+    q = np.empty((rows, K), np.int8)
+    sc = np.empty(rows, np.float32)
+    lib().sqo_quant_bulk(_p(x), _dt(x), rows, K, _p(keep), _p(q), _p(sc))
+    return q, sc
+
+
+def gather_columns(x: np.ndarray, idx: np.ndarray, ld: int | None = None) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    ld = idx.shape[0] if ld is None else ld
+    out = np.empty((rows, ld), np.float32)
+    lib().sqo_gather_columns(_p(x), _dt(x), rows, K, _p(idx), idx.shape[0], ld, _p(out))
+    return out
+
+
+def dequant_split(acc, x_scale, w_scale, x_out, w_out, n: int | None = None):
+    """-> (y float32, y bf16 bits, magnitude |Y_bulk| + sum |x_out w_out| fp64)."""
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    x_scale = np.ascontiguousarray(x_scale, dtype=np.float32)
+    w_scale = np.ascontiguousarray(w_scale, dtype=np.float32)
+    x_out = np.ascontiguousarray(x_out, dtype=np.float32)
+    w_out = np.ascontiguousarray(w_out, dtype=np.float32)
+    M, N = acc.shape
+    ld = x_out.shape[1]
+    assert w_out.shape == (N, ld) and x_out.shape[0] == M
+    n = ld if n is None else n
+    y = np.empty((M, N), np.float32)
+    yb = np.empty((M, N), np.uint16)
+    mag = np.empty((M, N), np.float64)
+    lib().sqo_dequant_split(_p(acc), _p(x_scale), _p(w_scale), M, N, _p(x_out), _p(w_out), n, ld,
+                            _p(y), _p(yb), _p(mag))
+    return y, yb, mag
+
+
+def linear_split(x: np.ndarray, w: np.ndarray, threshold: float, calib: list | None = None):
+    """The decomposed layer on one batch: outlier set from the calibration
+    maxima of x, bulk int8 of x and w, outlier columns in fp32."""
+    xmax = np.zeros(x.shape[1], np.float32)
+    for b in (calib if calib is not None else [x]):
+        col_absmax(b, xmax)
+    keep, idx = outlier_split(xmax, threshold)
+    wq, w_scale = quant_bulk(w, keep)
+    xq, x_scale = quant_bulk(x, keep)
+    x_out = gather_columns(x, idx)
+    w_out = gather_columns(w, idx)
+    acc = gemm_i8(xq, wq)
+    y, yb, mag = dequant_split(acc, x_scale, w_scale, x_out, w_out)
+    return dict(xmax=xmax, keep=keep, idx=idx, wq=wq, w_scale=w_scale, xq=xq, x_scale=x_scale,
+                x_out=x_out, w_out=w_out, acc=acc, y=y, y_bf16=yb, mag=mag)
+
+
+def alpha_search(x: np.ndarray, w: np.ndarray, alphas, eps: float = 1e-8, calib: list | None = None):
+    """W8A8 relative output error ||Yq - Y||_F / ||Y||_F of the fp32 path for
+    each alpha (Y = X W^T in fp64) -> (errors list, best alpha). Ties go to
+    the first alpha listed."""
+    xf = x.astype(np.float64) if x.dtype != np.uint16 else _bf16_bits_to_f64(x)
+    wf = w.astype(np.float64) if w.dtype != np.uint16 else _bf16_bits_to_f64(w)
+    Y = matmul_xwT_f64(xf, wf)
+    errs = []
+    for a in alphas:
+        out = linear(x, w, a, eps, calib)
+        errs.append(rel_frobenius_f64(out["y"].astype(np.float64), Y))
+    best = int(np.argmin(errs))
+    return errs, alphas[best]
+
+
+def _bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def e4m3_to_f64(b: np.ndarray) -> np.ndarray:
+    f = np.vectorize(lambda v: lib().sqo_e4m3_to_f64(int(v)), otypes=[np.float64])
+    return f(np.asarray(b, dtype=np.uint8))
+
+
+def e4m3_from_f64(v: np.ndarray) -> np.ndarray:
+    f = np.vectorize(lambda x: lib().sqo_e4m3_from_f64(float(x)), otypes=[np.uint8])
+    return f(np.asarray(v, dtype=np.float64))
+
+
+def quant_row_e4m3(v: np.ndarray):
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    q = np.empty(v.shape[0], np.uint8)
+    s = np.zeros(1, np.float32)
+    lib().sqo_quant_row_e4m3(_p(v), v.shape[0], _p(q), _p(s))
+    return q, s[0]
+
+
+def quant_rows_e4m3_f64(v: np.ndarray):
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    q = np.empty(v.shape, np.uint8)
+    sc = np.empty(v.shape[0], np.float64)
+    lib().sqo_quant_rows_e4m3_f64(_p(v), v.shape[0], v.shape[1], _p(q), _p(sc))
+    return q, sc
+
+
+def w8a8_e4m3_error_f64(X: np.ndarray, W: np.ndarray) -> float:
+    """Relative output error with per-token FP8 E4M3 activations and
+    per-output-channel FP8 E4M3 weights, fp64."""
+    xq, sa = quant_rows_e4m3_f64(X)
+    wq, sw = quant_rows_e4m3_f64(W)
+    T, K = xq.shape
+    N = wq.shape[0]
+    Yq = np.empty((T, N), np.float64)
+    lib().sqo_w8a8_e4m3_f64(_p(xq), _p(sa), _p(wq), _p(sw), T, N, K, _p(Yq))
+    return rel_frobenius_f64(Yq, matmul_xwT_f64(X, W))
+
+
+def w8a8_per_tensor_error_f64(X: np.ndarray, W: np.ndarray) -> float:
+    """Relative output error with ONE activation scale for the whole tensor
+    (the per-row quantizer applied to the flattened tensor) and
+    per-output-channel weights, fp64."""
+    T, K = X.shape
+    xq, sa = quant_rows_f64(np.ascontiguousarray(X, dtype=np.float64).reshape(1, T * K))
+    wq, sw = quant_rows_f64(W)
+    N = wq.shape[0]
+    Yq = np.empty((T, N), np.float64)
+    lib().sqo_w8a8_f64(_p(xq.reshape(T, K)), _p(np.full(T, sa[0])), _p(wq), _p(sw), T, N, K, _p(Yq))
+    return rel_frobenius_f64(Yq, matmul_xwT_f64(X, W))

@@ -62,7 +62,13 @@ enum {
     MUT_SCALE_128 = 9,         /* scale = amax/128 (asymmetric range) */
     MUT_FOLD_DIVIDES = 10,     /* weights divided by s instead of multiplied */
     MUT_COLMAX_NO_ABS = 11,    /* column max of signed values, not magnitudes */
-    MUT_SMOOTH_WRONG_INDEX = 12 /* activation channel j divided by s[j+1] */
+    MUT_SMOOTH_WRONG_INDEX = 12, /* activation channel j divided by s[j+1] */
+    MUT_TENSOR_MAX_UNSMOOTHED = 13, /* per-tensor maximum taken before smoothing */
+    MUT_NORM_NO_EPS = 14,      /* RMSNorm without its epsilon */
+    MUT_NORM_MEAN_ABS = 15,    /* RMSNorm from the mean |x| instead of the mean square */
+    MUT_SPLIT_MAX_ALL = 16,    /* bulk scale taken over the outlier channels too */
+    MUT_SPLIT_DROP_OUTLIERS = 17, /* decomposition forgets the floating-point term */
+    MUT_E4M3_TRUNCATE = 18     /* FP8 E4M3 conversion truncates instead of rounding */
 };
 static int g_mutation = MUT_NONE;
 
@@ -450,6 +456,290 @@ double sqo_rel_frobenius_f64(const double *Yq, const double *Y, int64_t n)
         den += Y[i] * Y[i];
     }
     return sqrt(num) / sqrt(den);
+}
+
+/* ======================================================================
+ * Next steps on the same layer: other activation granularities, the norm
+ * fold, the outlier decomposition and the FP8 sibling. Same rules as above:
+ * direct loops over each definition, fp32 in the order written unless noted.
+ * ====================================================================== */
+
+/* ---- per-tensor activation scales (O2 dynamic, O3 static) ---------------- */
+
+/* Smoothed value of one activation: RN(x / s_j), or x itself when s is NULL
+ * (the unsmoothed layer). */
+static float smoothed(const void *x, int dt, int64_t i, const float *s, int64_t j)
+{
+    float v = load_elem(x, dt, i);
+    return s ? v / s[j] : v;
+}
+
+/* amax = max(amax, max_{t,j} |RN(X_tj / s_j)|) over a [rows x cols] batch: the
+ * single range a per-tensor scale must cover ([KJ] "The outlier structure": a
+ * symmetric per-tensor scale covers the largest absolute value present). Run
+ * on the batch being quantized it gives the dynamic per-tensor range (O2);
+ * accumulated over calibration batches it gives the frozen static range (O3,
+ * [KJ] "Static scaling"; [SQE] "Where it fits": O2 and O3). The caller
+ * initialises amax (+0 for a fresh range). */
+void sqo_tensor_absmax(const void *x, int dt, int64_t rows, int64_t cols, const float *s,
+                       float *amax)
+{
+    float m = *amax;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < cols; ++j) {
+            float v = (g_mutation == MUT_TENSOR_MAX_UNSMOOTHED) ? load_elem(x, dt, r * cols + j)
+                                                                : smoothed(x, dt, r * cols + j, s, j);
+            float a = fabsf(v);
+            if (a > m) m = a;
+        }
+    *amax = m;
+}
+
+/* Per-tensor symmetric int8 of the smoothed activations with a given range
+ * amax: scale = amax / 127 (1 for amax = 0), q = clamp(round(RN(X/s) / scale),
+ * -127, 127). With a static (calibrated) range the clamp is what happens to an
+ * input beyond it ([KJ] "Static scaling": such inputs are clipped; [OO] "The
+ * four operations"). Every x_scale[t] is set to the one scale, so the
+ * per-token epilogue of the GEMM applies it unchanged. */
+void sqo_quant_act_per_tensor(const void *x, int dt, int64_t T, int64_t K, const float *s,
+                              float amax, int8_t *xq, float *x_scale)
+{
+    const float scale = (amax == 0.0f) ? 1.0f : amax / 127.0f;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t j = 0; j < K; ++j)
+            xq[t * K + j] = (amax == 0.0f) ? 0 : code_of(smoothed(x, dt, t * K + j, s, j), scale, amax);
+        x_scale[t] = scale;
+    }
+}
+
+/* ---- RMSNorm with the smoothing folded into its gain ---------------------- */
+
+/* g'_j = RN(g_j / s_j): diag(s)^-1 folded into the norm's per-channel gain
+ * offline ([SQE] "Why the rescaling is free at runtime"; [II] "What
+ * SmoothQuant does": the 1/s_j folds into the preceding RMSNorm gain). */
+void sqo_fold_norm_gain(const void *g, int dt, int64_t K, const float *s, float *gf)
+{
+    for (int64_t j = 0; j < K; ++j) gf[j] = load_elem(g, dt, j) / s[j];
+}
+
+/* RMSNorm of one token row followed by the per-token quantizer:
+ *   r_t   = 1 / sqrt(sum_j x_tj^2 / K + eps), in fp64 (sum in index order),
+ *           rounded once to fp32
+ *   xh_tj = RN(RN(x_tj * r_t) * g'_j)          (fp32, the norm's output)
+ *   (xq[t, :], x_scale[t]) = dynamic symmetric int8 of xh_t
+ * The norm emits the smoothed activations directly, so the separate division
+ * by s disappears from the runtime ([SQE] "Why the rescaling is free at
+ * runtime"). If r_in is not NULL its r_t is used instead of the computed one;
+ * r_out (may be NULL) receives the r_t used. */
+void sqo_rmsnorm_quant_act(const void *x, int dt, int64_t T, int64_t K, const float *gf, float eps,
+                           const float *r_in, int8_t *xq, float *x_scale, float *r_out)
+{
+#pragma omp parallel
+    {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            float r;
+            if (r_in) {
+                r = r_in[t];
+            } else {
+                double ss = 0.0;
+                for (int64_t j = 0; j < K; ++j) {
+                    double v = (double)load_elem(x, dt, t * K + j);
+                    ss += (g_mutation == MUT_NORM_MEAN_ABS) ? fabs(v) : v * v;
+                }
+                double ms = ss / (double)K;
+                if (g_mutation == MUT_NORM_MEAN_ABS) ms = ms * ms;
+                if (g_mutation != MUT_NORM_NO_EPS) ms = ms + (double)eps;
+                r = (float)(1.0 / sqrt(ms));
+            }
+            for (int64_t j = 0; j < K; ++j) {
+                float v = load_elem(x, dt, t * K + j) * r;
+                row[j] = v * gf[j];
+            }
+            sqo_quant_row(row, K, xq + t * K, x_scale + t);
+            if (r_out) r_out[t] = r;
+        }
+        free(row);
+    }
+}
+
+/* ---- mixed-precision decomposition (LLM.int8()-style) --------------------- */
+
+/* Static outlier set from calibration maxima: channel j is an outlier when
+ * xmax_j >= threshold. keep[j] = 0 for outliers, 1 otherwise; idx receives the
+ * outlier channels in ascending order; returns their count ([MM]
+ * "Decomposition": a set determined once from calibration and stored with the
+ * checkpoint). */
+int64_t sqo_outlier_split(const float *xmax, int64_t K, float threshold, float *keep, int32_t *idx)
+{
+    int64_t n = 0;
+    for (int64_t j = 0; j < K; ++j) {
+        if (xmax[j] >= threshold) {
+            keep[j] = 0.0f;
+            idx[n++] = (int32_t)j;
+        } else {
+            keep[j] = 1.0f;
+        }
+    }
+    return n;
+}
+
+/* Per-row int8 of the bulk (non-outlier) channels: the row's scale covers the
+ * bulk only and the outlier channels get code 0, so an integer GEMM over the
+ * full K sums exactly the bulk terms ([MM] "Decomposition": the bulk
+ * quantization uses a scale chosen for the bulk distribution; [OO] "Route it,
+ * or move it"). Rows of X give per-token scales, rows of W per-output-channel
+ * scales. */
+void sqo_quant_bulk(const void *x, int dt, int64_t rows, int64_t K, const float *keep, int8_t *q,
+                    float *scale)
+{
+#pragma omp parallel
+    {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < rows; ++r) {
+            for (int64_t j = 0; j < K; ++j) {
+                float v = load_elem(x, dt, r * K + j);
+                row[j] = (keep[j] != 0.0f || g_mutation == MUT_SPLIT_MAX_ALL) ? v : 0.0f;
+            }
+            sqo_quant_row(row, K, q + r * K, scale + r);
+            if (g_mutation == MUT_SPLIT_MAX_ALL)
+                for (int64_t j = 0; j < K; ++j)
+                    if (keep[j] == 0.0f) q[r * K + j] = 0;
+        }
+        free(row);
+    }
+}
+
+/* out[r, o] = x[r, idx[o]] as fp32 for o < n, 0 for n <= o < ld: the outlier
+ * channels gathered into a dense [rows x ld] matrix. */
+void sqo_gather_columns(const void *x, int dt, int64_t rows, int64_t K, const int32_t *idx, int64_t n,
+                        int64_t ld, float *out)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t o = 0; o < ld; ++o)
+            out[r * ld + o] = (o < n) ? load_elem(x, dt, r * K + idx[o]) : 0.0f;
+}
+
+/* Y = Y_bulk + X_out W_out^T ([OO] "Route it, or move it": the sum over K
+ * splits into the int8 term and a thin floating-point term; [MM]
+ * "Decomposition"): Y_bulk = (float(acc) * sa_t) * sw_n as in the plain
+ * epilogue, the outlier term sum_o x_out[t,o] w_out[n,o] in fp64, their sum
+ * rounded once to fp32 (and that value to bf16). mag (may be NULL) receives
+ * |Y_bulk| + sum_o |x_out w_out|, the scale of the rounding error any fp32
+ * evaluation order makes. */
+void sqo_dequant_split(const int32_t *acc, const float *x_scale, const float *w_scale, int64_t M,
+                       int64_t N, const float *x_out, const float *w_out, int64_t n, int64_t ld,
+                       float *y_f32, uint16_t *y_bf16, double *mag)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; ++t) {
+        for (int64_t c = 0; c < N; ++c) {
+            float yb = ((float)acc[t * N + c] * x_scale[t]) * w_scale[c];
+            double yo = 0.0, mo = 0.0;
+            for (int64_t o = 0; o < n; ++o) {
+                double p = (double)x_out[t * ld + o] * (double)w_out[c * ld + o];
+                yo += p;
+                mo += fabs(p);
+            }
+            if (g_mutation == MUT_SPLIT_DROP_OUTLIERS) yo = 0.0;
+            float y = (float)((double)yb + yo);
+            if (y_f32) y_f32[t * N + c] = y;
+            if (y_bf16) y_bf16[t * N + c] = sqo_f32_to_bf16_rne(y);
+            if (mag) mag[t * N + c] = fabs((double)yb) + mo;
+        }
+    }
+}
+
+/* ---- FP8 E4M3 sibling ------------------------------------------------------ */
+
+/* E4M3 (the OCP "fn" variant: 4 exponent bits, bias 7, 3 mantissa bits, no
+ * infinities, largest finite 448, subnormal step 2^-9). Decoding a byte: */
+double sqo_e4m3_to_f64(uint8_t b)
+{
+    int sign = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Encoding with round to nearest, ties to even, saturating to +-448 (values
+ * beyond the largest finite code take it; there is no infinity). The sign
+ * of zero is kept. */
+uint8_t sqo_e4m3_from_f64(double v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    double a = fabs(v);
+    double q;
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {
+        q = ldexp(1.0, -9);                 /* subnormal quantum */
+    } else {
+        int e;
+        frexp(a, &e);                       /* a = f * 2^e, f in [0.5, 1) */
+        q = ldexp(1.0, e - 1 - 3);          /* 3 mantissa bits below the leading one */
+    }
+    double k = (g_mutation == MUT_E4M3_TRUNCATE) ? floor(a / q) : nearbyint(a / q);
+    double r = k * q;                       /* exact: k < 2^5, q a power of two */
+    if (r >= 448.0) return sign | 0x7E;
+    if (r == 0.0) return sign;
+    if (r < ldexp(1.0, -6)) return sign | (uint8_t)(r / ldexp(1.0, -9));
+    int e;
+    double f = frexp(r, &e);                /* r = f * 2^e */
+    int exp_field = e - 1 + 7;
+    int mant = (int)((f * 2.0 - 1.0) * 8.0);
+    return sign | (uint8_t)(exp_field << 3) | (uint8_t)mant;
+}
+
+/* Per-row FP8 quantization: scale = amax / 448 (1 for an all-zero row),
+ * code_j = E4M3(RN(v_j / scale)), the fp32 quotient encoded as above ([II]
+ * "The reversal condition is the format": per-token FP8 activations; the
+ * same per-row rule gives per-output-channel FP8 weights). */
+void sqo_quant_row_e4m3(const float *v, int64_t K, uint8_t *q, float *scale_out)
+{
+    float amax = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+        float a = fabsf(v[j]);
+        if (a > amax) amax = a;
+    }
+    float scale = (amax == 0.0f) ? 1.0f : amax / 448.0f;
+    for (int64_t j = 0; j < K; ++j) q[j] = sqo_e4m3_from_f64((double)(v[j] / scale));
+    *scale_out = scale;
+}
+
+/* The same rule in fp64 for the error experiments. */
+void sqo_quant_rows_e4m3_f64(const double *v, int64_t rows, int64_t K, uint8_t *q, double *scale)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *x = v + r * K;
+        double amax = 0.0;
+        for (int64_t j = 0; j < K; ++j)
+            if (fabs(x[j]) > amax) amax = fabs(x[j]);
+        double sc = (amax == 0.0) ? 1.0 : amax / 448.0;
+        for (int64_t j = 0; j < K; ++j) q[r * K + j] = sqo_e4m3_from_f64(x[j] / sc);
+        scale[r] = sc;
+    }
+}
+
+/* Yq[t, n] = (sum_k dec(xq[t,k]) dec(wq[n,k])) * sa[t] * sw[n] in fp64 (each
+ * product of two E4M3 values is exact in fp64; the sum runs in index order). */
+void sqo_w8a8_e4m3_f64(const uint8_t *xq, const double *sa, const uint8_t *wq, const double *sw,
+                       int64_t T, int64_t N, int64_t K, double *Yq)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += sqo_e4m3_to_f64(xq[t * K + k]) * sqo_e4m3_to_f64(wq[n * K + k]);
+            Yq[t * N + n] = acc * sa[t] * sw[n];
+        }
 }
 
 /* Thread count the OpenMP regions use (reported with CPU timings). */

@@ -312,6 +312,151 @@ def pin_dequant_epilogue():
     assert tyb.tolist() == [[0x3F80, 0x3F82, 0xBF80]], [hex(v) for v in tyb[0]]
 
 
+# ------------------------------------------------- next steps on the layer
+def _exact_smoothed(x, s_j):
+    return rn32(Fraction(float(x)) / Fraction(float(s_j)))
+
+
+def pin_per_tensor_scales():
+    """Per-tensor range = max over the whole batch of |rn32(x / s_j)| (exact
+    rationals); codes = clamp(rne(rn32(rn32(x/s_j) / rn32(amax/127)))), one
+    scale for every token; a static range clips a later batch that exceeds it
+    to +-127; a zero range gives scale 1 and codes 0."""
+    rng = np.random.default_rng(21)
+    T, K = 5, 48
+    x = rng.normal(size=(T, K)).astype(np.float32)
+    x[3, 7] = -9.75
+    s = rng.uniform(0.3, 3.0, K).astype(np.float32)
+    s[7] = 0.37
+    exact = max(abs(Fraction(float(_exact_smoothed(x[t, j], s[j])))) for t in range(T) for j in range(K))
+    amax = oracle.tensor_absmax(x, s)
+    assert _bits(amax) == _bits(np.float32(float(exact))), (amax, float(exact))
+    # running over batches = over their union
+    a1 = oracle.tensor_absmax(x[:2], s)
+    assert _bits(oracle.tensor_absmax(x[2:], s, a1)) == _bits(amax)
+    # no smoothing: plain max |x|
+    assert float(oracle.tensor_absmax(x, None)) == float(np.abs(x).max())
+    xq, xs = oracle.quant_act_per_tensor(x, s, amax)
+    scale = rn32(Fraction(float(amax)) / 127)
+    assert all(_bits(v) == _bits(scale) for v in xs), xs
+    fs = Fraction(float(scale))
+    for t in range(T):
+        for j in range(K):
+            e = max(-127, min(127, rne_int(Fraction(float(rn32(Fraction(float(_exact_smoothed(x[t, j], s[j]))) / fs))))))
+            assert int(xq[t, j]) == e, (t, j, int(xq[t, j]), e)
+    # static range from a calibration batch, applied to a larger batch: clipped
+    big = (x * 3).astype(np.float32)
+    bq, _ = oracle.quant_act_per_tensor(big, s, amax)
+    assert int(bq[3, 7]) == -127 and int(bq.max()) <= 127 and int(bq.min()) >= -127
+    hot = np.abs(np.array([[float(_exact_smoothed(big[t, j], s[j])) for j in range(K)] for t in range(T)]))
+    assert (np.abs(bq[hot > 127.5 * float(scale)]) == 127).all()
+    zq, zs = oracle.quant_act_per_tensor(np.zeros((2, 16), np.float32), None, 0.0)
+    assert not zq.any() and (zs == 1.0).all()
+
+
+def pin_norm_fold():
+    """Folded gain g'_j = rn32(g_j / s_j) (exact rationals). RMSNorm factor r_t
+    = fp32 of torch.nn.functional.rms_norm(x)_j / x_j in fp64 (a library
+    routine), to 1 ulp, with eps large enough to matter; codes and scale equal
+    the exact-rational evaluation of rn32(rn32(x r_t) g'_j) followed by the
+    per-token quantizer; a power-of-two rescaling of the input leaves the codes
+    unchanged; an all-zero row gives scale 1 and codes 0."""
+    import torch
+    rng = np.random.default_rng(22)
+    T, K = 4, 64
+    x = rng.normal(size=(T, K)).astype(np.float32)
+    x[:, 5] *= 40.0
+    x[3] = 0.0
+    g = rng.uniform(0.5, 1.5, K).astype(np.float32)
+    s = rng.uniform(0.2, 4.0, K).astype(np.float32)
+    gf = oracle.fold_norm_gain(g, s)
+    for j in range(K):
+        assert _bits(gf[j]) == _bits(rn32(Fraction(float(g[j])) / Fraction(float(s[j])))), j
+    eps = 0.25
+    xq, xs, r = oracle.rmsnorm_quant_act(x, gf, eps)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x.astype(np.float64)), (K,), eps=eps).numpy()
+    for t in range(T - 1):
+        rt = ref[t, 0] / float(x[t, 0])
+        assert abs(float(r[t]) - rt) <= ulp32(rt), (t, float(r[t]), rt)
+    assert abs(float(r[T - 1]) - 1.0 / math.sqrt(eps)) <= ulp32(2.0)
+    for t in range(T):
+        xh = [rn32(Fraction(float(rn32(Fraction(float(x[t, j])) * Fraction(float(r[t]))))) * Fraction(float(gf[j])))
+              for j in range(K)]
+        eq, esc = exact_quant_row(np.array(xh, np.float32))
+        assert _bits(xs[t]) == _bits(esc), (t, xs[t], esc)
+        assert np.array_equal(xq[t], eq), (t, np.nonzero(xq[t] != eq))
+    assert not xq[T - 1].any() and float(xs[T - 1]) == 1.0
+    q4, s4, _ = oracle.rmsnorm_quant_act((x * 4).astype(np.float32), gf, 1e-30)
+    q1, s1, _ = oracle.rmsnorm_quant_act(x, gf, 1e-30)
+    assert np.array_equal(q4[:T - 1], q1[:T - 1]) and np.array_equal(s4[:T - 1], s1[:T - 1])
+    # a given r_t replaces the computed one
+    qr, _, rr = oracle.rmsnorm_quant_act(x, gf, eps, r_in=r * 2)
+    assert np.array_equal(rr, r * 2)
+
+
+def pin_decomposition_exact():
+    """Bulk channels on the integer grid with a 127 in every row, so the bulk
+    quantization is lossless only if its scale ignores the outlier channels;
+    outlier channels far off the grid. The decomposed layer then equals the
+    exact product X W^T rounded once to fp32 (exact rationals), and the
+    outlier set is exactly the channels at or above the threshold."""
+    rng = np.random.default_rng(23)
+    M, N, K = 4, 6, 32
+    out_ch = [3, 17, 30]
+    x = rng.integers(-127, 128, (M, K)).astype(np.float32)
+    w = rng.integers(-127, 128, (N, K)).astype(np.float32)
+    x[:, 0] = 127.0
+    w[:, 1] = -127.0
+    x[:, out_ch] = rng.uniform(200.0, 1000.0, (M, 3)).astype(np.float32) + np.float32(0.375)
+    w[:, out_ch] = rng.normal(size=(N, 3)).astype(np.float32)
+    xmax = oracle.col_absmax(x)
+    keep, idx = oracle.outlier_split(xmax, 150.0)
+    assert idx.tolist() == out_ch and keep.tolist() == [0.0 if j in out_ch else 1.0 for j in range(K)]
+    res = oracle.linear_split(x, w, 150.0)
+    assert (res["x_scale"] == 1.0).all() and (res["w_scale"] == 1.0).all()
+    assert not res["xq"][:, out_ch].any() and not res["wq"][:, out_ch].any()
+    for t in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(x[t, k])) * Fraction(float(w[n, k])) for k in range(K))
+            assert _bits(res["y"][t, n]) == _bits(rn32(exact)), (t, n, res["y"][t, n], float(exact))
+    # the worked example with the outlier routed out: the bulk scale covers values below 1
+    g = golden("worked_example_outlier_30.json")
+    row = np.full(64, 0.9, np.float32)
+    row[17] = g["outlier"]
+    row[100 % 64] = 0.5
+    kp, _ = oracle.outlier_split(np.abs(row), 6.0)
+    q, sc = oracle.quant_bulk(row[None, :], kp)
+    assert _bits(sc[0]) == _bits(rn32(Fraction(float(np.float32(0.9))) / 127))
+    assert int(q[0, 17]) == 0 and int(q[0, 36]) == rne_int(Fraction(float(rn32(Fraction(1, 2) / Fraction(float(sc[0]))))))
+
+
+def pin_e4m3_codes():
+    """FP8 E4M3 (no infinities, largest 448): decoding every byte and encoding
+    every representable value, every midpoint between neighbours (ties to the
+    even code) and random values agree with torch.float8_e4m3fn (a library
+    conversion); values beyond 448 saturate; the per-row FP8 quantizer's
+    largest element encodes as 448."""
+    import torch
+    allb = np.arange(256, dtype=np.uint8)
+    dec = oracle.e4m3_to_f64(allb)
+    tdec = torch.from_numpy(allb).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    fin = ~np.isnan(tdec)
+    assert np.array_equal(np.isnan(dec), ~fin)
+    assert np.array_equal(dec[fin], tdec[fin])
+    pos = np.unique(dec[fin & (dec >= 0)])
+    mids = (pos[1:] + pos[:-1]) / 2
+    rng = np.random.default_rng(24)
+    vals = np.concatenate([pos, -pos, mids, -mids, rng.uniform(-448, 448, 2000),
+                           rng.normal(size=500) * 1e-2, np.array([-0.0, 0.0])])
+    ours = oracle.e4m3_from_f64(vals)
+    theirs = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    bad = np.nonzero(ours != theirs)[0]
+    assert bad.size == 0, [(vals[i], int(ours[i]), int(theirs[i])) for i in bad[:5]]
+    assert oracle.e4m3_from_f64(np.array([449.0, 470.0, 1e9, -1e9])).tolist() == [0x7E, 0x7E, 0x7E, 0xFE]
+    q, sc = oracle.quant_row_e4m3(np.array([0.5, -3.0, 1.0, 0.0], np.float32))
+    assert _bits(sc) == _bits(rn32(Fraction(3) / 448)) and int(q[1]) == 0xFE
+
+
 FAST_PINS = [
     pin_worked_example,
     pin_ties_half_even,
@@ -326,4 +471,8 @@ FAST_PINS = [
     pin_reconstruction_bounds,
     pin_gemm_bruteforce,
     pin_dequant_epilogue,
+    pin_per_tensor_scales,
+    pin_norm_fold,
+    pin_decomposition_exact,
+    pin_e4m3_codes,
 ]

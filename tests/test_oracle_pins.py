@@ -96,3 +96,48 @@ def test_fp32_chain_reproduces_experiment(experiment, oracle_lib):
     d = g["printed_decimals"]
     assert round(errs[0], d) == g["w8a8_rel_error_before"], errs
     assert round(errs[1], d) == g["w8a8_rel_error_after"], errs
+
+
+def _smoothed_experiment(X, W):
+    s = oracle.smooth_factors_f64(oracle.col_absmax_f64(X), oracle.col_absmax_f64(W), 0.5)
+    return oracle.smooth_f64(X, W, s)
+
+
+def test_per_tensor_and_fp8_errors(experiment, oracle_lib):
+    """Same data: per-tensor INT8 activations 21% -> 2.9% with smoothing, per-
+    token FP8 E4M3 activations (and FP8 weights) 3.3% -> 2.9%."""
+    g = pins.golden("format_and_granularity.json")
+    X, W, _ = experiment
+    Xs, Ws = _smoothed_experiment(X, W)
+    assert round(100 * oracle.w8a8_per_tensor_error_f64(X, W)) == g["per_tensor_int8_percent_before"]
+    assert round(100 * oracle.w8a8_per_tensor_error_f64(Xs, Ws), 1) == g["per_tensor_int8_percent_after"]
+    assert round(100 * oracle.w8a8_e4m3_error_f64(X, W), 1) == g["per_token_fp8_percent_before"]
+    assert round(100 * oracle.w8a8_e4m3_error_f64(Xs, Ws), 1) == g["per_token_fp8_percent_after"]
+
+
+def test_per_tensor_fp32_chain(experiment, oracle_lib):
+    """The fp32 per-tensor path (range of the smoothed batch, one scale, the
+    int8 GEMM and epilogue) gives the printed 21% and 2.9% on the same data."""
+    g = pins.golden("format_and_granularity.json")
+    X, W, Y = experiment
+    X32, W32 = X.astype(np.float32), W.astype(np.float32)
+    errs = []
+    for s in (None, oracle.smooth_factors(oracle.col_absmax(X32), oracle.col_absmax(W32), 0.5)):
+        ones = np.ones(X.shape[1], np.float32)
+        wq, sw = oracle.fold_quant_weights(W32, ones if s is None else s)
+        xq, sa = oracle.quant_act_per_tensor(X32, s, oracle.tensor_absmax(X32, s))
+        y, _ = oracle.dequant(oracle.gemm_i8(xq, wq), sa, sw)
+        errs.append(100 * oracle.rel_frobenius_f64(y.astype(np.float64), Y))
+    assert round(errs[0]) == g["per_tensor_int8_percent_before"], errs
+    assert round(errs[1], 1) == g["per_tensor_int8_percent_after"], errs
+
+
+def test_alpha_search_fp32_path(experiment, oracle_lib):
+    """The alpha search over the table's alphas, on the fp32 path fed fp32
+    data: the table's error percentages and the minimum at alpha = 0.5."""
+    g = pins.golden("outlier_experiment.json")
+    X, W, _ = experiment
+    alphas = [row["alpha"] for row in g["alpha_table"]]
+    errs, best = oracle.alpha_search(X.astype(np.float32), W.astype(np.float32), alphas)
+    assert [round(100 * e, 1) for e in errs] == [row["error_percent"] for row in g["alpha_table"]], errs
+    assert best == 0.5
