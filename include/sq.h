@@ -129,6 +129,68 @@ sq_status sq_smooth_quant_act(const void* x, sq_dtype dt, int64_t T, int64_t K,
                               const float* s, int8_t* xq, float* x_scale,
                               sq_stream_t stream);
 
+/* ---------------------------------------------------------------- per-tensor scales (O2, O3)
+ * One activation scale for the whole tensor instead of one per token: the
+ * per-tensor dynamic (O2) and per-tensor static (O3) levels of "SmoothQuant
+ * Explained", "Where it fits, and where it does not". Static scales are
+ * frozen at calibration and clip any later input beyond them; dynamic scales
+ * cost a reduction over the tensor before every quantized matmul ("Why are
+ * activations harder to quantize than weights in a transformer?", "Static
+ * scaling" / "Dynamic scaling").
+ *
+ * sq_tensor_absmax: running per-tensor range of the smoothed activations,
+ *   amax[0] = max(amax[0], max_{r,j} |RN(x[r, j] / s_j)|)
+ *   x     [rows x cols], dtype dt (SQ_F32 or SQ_BF16), device.
+ *   s     [cols] float, device, every s_j positive and finite; or NULL for the
+ *         unsmoothed tensor (the maximum of |x|).
+ *   amax  [1] float, device, in/out; the caller sets it to +0 for a fresh
+ *         range. On the batch about to be quantized it gives the O2 range;
+ *         accumulated over calibration batches (or applied once to the [1 x K]
+ *         calibration maxima xmax) it gives the O3 range.
+ *   Exact: the division is monotone, so each column's maximum is divided once.
+ *
+ * sq_quant_act_per_tensor: codes with one scale,
+ *   scale   = amax[0] / 127                                  (1.0 if amax[0] == 0)
+ *   xq_tj   = clamp(round(RN(x_tj / s_j) / scale), -127, 127)
+ *   x_scale_t = scale for every t, so sq_w8a8_gemm applies it unchanged.
+ *   x [T x K] (SQ_F32 or SQ_BF16), s [K] or NULL, amax [1] float (read on the
+ *   device), xq [T x K] int8 out, x_scale [T] float out: all device.
+ *   Values beyond the range clamp to +-127 (the static-scale clipping). */
+sq_status sq_tensor_absmax(const void* x, sq_dtype dt, int64_t rows, int64_t cols,
+                           const float* s, float* amax, sq_stream_t stream);
+sq_status sq_quant_act_per_tensor(const void* x, sq_dtype dt, int64_t T, int64_t K,
+                                  const float* s, const float* amax, int8_t* xq,
+                                  float* x_scale, sq_stream_t stream);
+
+/* ---------------------------------------------------------------- RMSNorm with the folded gain
+ * The deployed form of step a4: diag(s)^-1 folded offline into the gain of
+ * the RMSNorm that feeds the layer, so the norm itself emits the smoothed
+ * activations ("SmoothQuant Explained", "Why the rescaling is free at
+ * runtime"; "Why do activation outliers break INT8 W8A8...", "A strong
+ * answer": the 1/s_j folds into the preceding RMSNorm gain).
+ *
+ * sq_fold_norm_gain (offline):  gain_folded_j = RN(gain_j / s_j)
+ *   gain [K] dtype dt (SQ_F32 or SQ_BF16), s [K] float, gain_folded [K] float out.
+ *
+ * sq_rmsnorm_quant_act: per token row t
+ *   r_t     = RN32(1 / sqrt(sum_j x_tj^2 / K + eps))   (fp64 sum and 1/sqrt)
+ *   v_tj    = RN(RN(x_tj * r_t) * gain_folded_j)       (the norm output, fp32)
+ *   x_scale_t = max_j |v_tj| / 127 (1.0 for an all-zero row),
+ *   xq_tj   = clamp(round(v_tj / x_scale_t), -127, 127)
+ *   x [T x K] (SQ_F32 or SQ_BF16), gain_folded [K] float, xq [T x K] int8 out,
+ *   x_scale [T] float out, inv_rms [T] float out (r_t) or NULL: all device.
+ *   eps > 0 (the norm's epsilon). K <= 32768 for SQ_BF16 input, K <= 16384 for
+ *   SQ_F32 (the row is held in registers); larger K returns SQ_ERR_UNSUPPORTED.
+ *   The norm output is quantized from fp32; it is never rounded to bf16.
+ *   The sum of squares is exact per term but its fp64 rounding order is the
+ *   kernel's, so r_t may differ from an index-order evaluation in the last
+ *   fp32 bit in rare cases; everything after r_t is exact. */
+sq_status sq_fold_norm_gain(const void* gain, sq_dtype dt, int64_t K, const float* s,
+                            float* gain_folded, sq_stream_t stream);
+sq_status sq_rmsnorm_quant_act(const void* x, sq_dtype dt, int64_t T, int64_t K,
+                               const float* gain_folded, float eps, int8_t* xq,
+                               float* x_scale, float* inv_rms, sq_stream_t stream);
+
 /* ---------------------------------------------------------------- step a5
  * int8 x int8 -> int32 GEMM with the dequantizing epilogue.
  *   acc_tn = sum_k xq_tk * wq_nk                        (exact int32)
@@ -152,6 +214,58 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* x_scale, const int8_t* wq,
                        const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
                        sq_dtype out_dt, void* workspace, size_t ws_bytes,
                        sq_stream_t stream);
+
+/* ---------------------------------------------------------------- mixed-precision decomposition
+ * The LLM.int8()-style alternative to smoothing: a static set of outlier
+ * input channels keeps full precision and the rest of the contraction runs
+ * in int8. The sum over K splits exactly,
+ *   Y = X_bulk W_bulk^T + X_out W_out^T,
+ * so the only error is that of the bulk quantization, whose scales no longer
+ * have to cover the outliers ("Activation Outlier Channels and Mixed-Precision
+ * Decomposition", "Decomposition: keep the outliers in high precision"; "One
+ * outlier" notes, "Route it, or move it"). The set is chosen once from
+ * calibration maxima, so the kernels can specialize on it (same page: a set
+ * determined once from calibration and stored with the checkpoint).
+ *
+ * sq_outlier_split: channel j is an outlier when xmax[j] >= threshold.
+ *   xmax [K] float (from sq_calibrate_absmax); keep [K] float out (0 for an
+ *   outlier, 1 otherwise); idx [K] int32 out (capacity K), the outlier channels
+ *   in ascending order; count [1] int32 out, their number. All device.
+ *
+ * sq_quant_bulk: per-row int8 of the bulk channels,
+ *   scale_r = max_{j: keep_j = 1} |x_rj| / 127   (1.0 if that is 0)
+ *   q_rj    = clamp(round(x_rj / scale_r), -127, 127) for bulk channels, 0 for
+ *             outlier channels.
+ *   Rows of X give per-token scales, rows of W per-output-channel scales.
+ *   x [rows x K] (SQ_F32 or SQ_BF16), keep [K] float with every entry exactly 0
+ *   or 1, q [rows x K] int8 out, scale [rows] float out: all device.
+ *
+ * sq_gather_columns: out[r, o] = float(x[r, idx[o]]) for o < n, 0 for
+ *   n <= o < ld. x [rows x K] (SQ_F32 or SQ_BF16), idx [n] int32 with entries
+ *   in [0, K) (an entry outside reads nothing and gives NaN), out [rows x ld]
+ *   float: device. For the outlier operands x_out and w_out below.
+ *
+ * sq_w8a8_gemm_split: the int8 GEMM of sq_w8a8_gemm over the full K (the
+ *   outlier channels hold code 0) plus the outlier term in its epilogue,
+ *     y_tn = fma chain over o = 0 .. ld-1 of x_out[t, o] * w_out[n, o],
+ *            starting from (float(acc_tn) * x_scale_t) * w_scale_n,
+ *   every step an fp32 fused multiply-add, then rounded to out_dt.
+ *   x_out [M x ld] and w_out [N x ld] float, device, 16-byte aligned, zero
+ *   beyond the real outlier count; ld a multiple of 4 in [0, 64] (ld = 0 is
+ *   the plain GEMM). out_dt SQ_F32 or SQ_BF16. Workspace and every other
+ *   argument as for sq_w8a8_gemm. */
+sq_status sq_outlier_split(const float* xmax, int64_t K, float threshold, float* keep,
+                           int32_t* idx, int32_t* count, sq_stream_t stream);
+sq_status sq_quant_bulk(const void* x, sq_dtype dt, int64_t rows, int64_t K, const float* keep,
+                        int8_t* q, float* scale, sq_stream_t stream);
+sq_status sq_gather_columns(const void* x, sq_dtype dt, int64_t rows, int64_t K,
+                            const int32_t* idx, int64_t n, int64_t ld, float* out,
+                            sq_stream_t stream);
+sq_status sq_w8a8_gemm_split(const int8_t* xq, const float* x_scale, const int8_t* wq,
+                             const float* w_scale, int64_t M, int64_t N, int64_t K,
+                             const float* x_out, const float* w_out, int64_t ld, void* y,
+                             sq_dtype out_dt, void* workspace, size_t ws_bytes,
+                             sq_stream_t stream);
 
 /* ---------------------------------------------------------------- no-alloc decode GEMM
  * The pages have no counterpart to this entry point; it exists for callers
@@ -177,6 +291,33 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* x_scale, const int8_t* wq,
 sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* x_scale, const int8_t* wq,
                                const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
                                sq_dtype out_dt, sq_stream_t stream);
+
+/* ---------------------------------------------------------------- alpha search
+ * Per-layer choice of the migration strength: for each candidate alpha the
+ * whole path (a2 smoothing factors, a3 fold + quantize W, a4 smooth + quantize
+ * X, a5 GEMM with fp32 output) runs on the calibration batch x, and its
+ * relative output error
+ *   err[a] = ||Yq(alpha_a) - Y||_F / ||Y||_F,   Y = X W^T
+ * is returned ("Why do activation outliers break INT8 W8A8...", "A strong
+ * answer": the alpha sweep and its W8A8 error column; "SmoothQuant
+ * Explained", "Alpha: how much difficulty to move": the best alpha is
+ * model-specific). The maxima (a1) come from x and w once. Y is computed once
+ * with cuBLAS (a plain floating-point GEMM: bf16 or fp32 operands, fp32
+ * accumulation); the sums of squares are fp64.
+ *   x [T x K], w [N x K]: dtype in_dt (SQ_F32 or SQ_BF16), device.
+ *   alphas [n_alpha] float, HOST, each in [0, 1]; 1 <= n_alpha <= 64.
+ *   eps as for sq_smooth_factors.
+ *   err [n_alpha] double, HOST, out. best_alpha [1] float, HOST, out (the first
+ *   alpha with the smallest error), or NULL.
+ *   workspace: device, ws_bytes >= sq_alpha_search_workspace_size(T, N, K,
+ *   n_alpha), zero-filled before its first use (it holds a GEMM workspace).
+ * The call synchronizes `stream` before it returns (the errors are host
+ * values). */
+size_t sq_alpha_search_workspace_size(int64_t T, int64_t N, int64_t K, int64_t n_alpha);
+sq_status sq_alpha_search(const void* x, const void* w, sq_dtype in_dt, int64_t T, int64_t N,
+                          int64_t K, const float* alphas, int64_t n_alpha, float eps,
+                          double* err, float* best_alpha, void* workspace, size_t ws_bytes,
+                          sq_stream_t stream);
 
 /* ---------------------------------------------------------------- whole layer
  * The whole path on one batch: calibrate X and W (a1, from zero), smoothing

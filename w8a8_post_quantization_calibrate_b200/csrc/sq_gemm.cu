@@ -60,6 +60,7 @@ constexpr uint32_t IDESC_STREAM = make_idesc_i8(S_BM, S_BN);
 constexpr int STREAM_MAX_M = 16;
 
 enum OutKind { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
+constexpr int kMaxSplitLd = 64;  // outlier channels the decomposed epilogue takes
 
 constexpr size_t tiled_smem_bytes() {
     return 1024 /*alignment slack*/ + STAGES * (A_STAGE + B_STAGE) + 256 /*barriers etc*/;
@@ -80,10 +81,59 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
     nb = idx / gm;
 }
 
+// The floating-point term of the mixed-precision decomposition ("Activation
+// Outlier Channels and Mixed-Precision Decomposition", "Decomposition"; "One
+// outlier" notes, "Route it, or move it"): the few outlier input channels,
+// gathered into x_out [M x ld] and w_out [N x ld] (fp32, zero-padded to ld, a
+// multiple of 4), are added to the dequantized int8 term in the epilogue as a
+// chain of fp32 fused multiply-adds in channel order:
+//   y = fma(x_out[ld-1], w_out[ld-1], ... fma(x_out[0], w_out[0], y_bulk)).
+struct SplitTerm {
+    const float* x_out = nullptr;
+    const float* w_out = nullptr;
+    int ld = 0;
+};
+
+// v[i] += sum_o x_out[row, o] * w_out[col0 + i, o] for the 32 columns of a row.
+// All lanes of a warp read the same w_out element at once (a broadcast).
+__device__ __forceinline__ void add_split32(float (&v)[32], int64_t row, int col0, int N, const SplitTerm& sp) {
+    const float* xr = sp.x_out + row * (int64_t)sp.ld;
+#pragma unroll 1
+    for (int o = 0; o < sp.ld; o += 4) {
+        const float4 xo = __ldg(reinterpret_cast<const float4*>(xr + o));
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (col0 + i < N) {
+                const float4 wo = __ldg(reinterpret_cast<const float4*>(sp.w_out + (int64_t)(col0 + i) * sp.ld + o));
+                v[i] = fmaf(xo.x, wo.x, v[i]);
+                v[i] = fmaf(xo.y, wo.y, v[i]);
+                v[i] = fmaf(xo.z, wo.z, v[i]);
+                v[i] = fmaf(xo.w, wo.w, v[i]);
+            }
+        }
+    }
+}
+
+// The same sum for one output element (token t, output channel n).
+__device__ __forceinline__ float add_split1(float v, int64_t t, int64_t n, const SplitTerm& sp) {
+    const float* xr = sp.x_out + t * (int64_t)sp.ld;
+    const float* wr = sp.w_out + n * (int64_t)sp.ld;
+#pragma unroll 1
+    for (int o = 0; o < sp.ld; o += 4) {
+        const float4 xo = __ldg(reinterpret_cast<const float4*>(xr + o));
+        const float4 wo = __ldg(reinterpret_cast<const float4*>(wr + o));
+        v = fmaf(xo.x, wo.x, v);
+        v = fmaf(xo.y, wo.y, v);
+        v = fmaf(xo.z, wo.z, v);
+        v = fmaf(xo.w, wo.w, v);
+    }
+    return v;
+}
+
 // Stores 32 consecutive outputs of one row (row-major y, row stride N).
-template <int OUT>
+template <int OUT, bool SPLIT>
 __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int N, const uint32_t (&r)[32],
-                                            float sa, const float* __restrict__ w_scale) {
+                                            float sa, const float* __restrict__ w_scale, const SplitTerm& sp) {
     const int64_t base = row * (int64_t)N + col0;
     const bool full = (col0 + 32 <= N);
     if (OUT == kOutI32) {
@@ -113,6 +163,7 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
         for (int i = 0; i < 32; ++i)
             v[i] = (col0 + i < N) ? dequant((int32_t)r[i], sa, __ldg(w_scale + col0 + i)) : 0.0f;
     }
+    if (SPLIT) add_split32(v, row, col0, N, sp);
     if (OUT == kOutF32) {
         float* yp = static_cast<float*>(y) + base;
         if (full && (N & 3) == 0) {
@@ -143,11 +194,11 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
 }
 
 // ================================================================== prefill
-template <int OUT>
+template <int OUT, bool SPLIT>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const float* __restrict__ x_scale, const float* __restrict__ w_scale,
-                  void* __restrict__ y, int M, int N, int K, long long wait_limit) {
+                  void* __restrict__ y, int M, int N, int K, const SplitTerm sp, long long wait_limit) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -282,8 +333,8 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
                 tmem_wait_ld();
                 const int col0 = nb * BN + c * 32;
-                if (row_ok && col0 < N) store_row32<OUT>(y, row, col0, N, r0, sa, w_scale);
-                if (row_ok && col0 + 32 < N) store_row32<OUT>(y, row, col0 + 32, N, r1, sa, w_scale);
+                if (row_ok && col0 < N) store_row32<OUT, SPLIT>(y, row, col0, N, r0, sa, w_scale, sp);
+                if (row_ok && col0 + 32 < N) store_row32<OUT, SPLIT>(y, row, col0 + 32, N, r1, sa, w_scale, sp);
             }
             tc_fence_before();
             __syncwarp();
@@ -375,11 +426,11 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "n"(NCOLS) : "memory");
 }
 
-template <int OUT>
+template <int OUT, bool SPLIT>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ x_scale, const float* __restrict__ w_scale,
-                 void* __restrict__ y, int M, int N, int K, long long wait_limit) {
+                 void* __restrict__ y, int M, int N, int K, const SplitTerm sp, long long wait_limit) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -525,8 +576,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
                 tmem_wait_ld();
                 const int col0 = nb * BN + c * 32;
-                if (row_ok && col0 < N) store_row32<OUT>(y, row, col0, N, r0, sa, w_scale);
-                if (row_ok && col0 + 32 < N) store_row32<OUT>(y, row, col0 + 32, N, r1, sa, w_scale);
+                if (row_ok && col0 < N) store_row32<OUT, SPLIT>(y, row, col0, N, r0, sa, w_scale, sp);
+                if (row_ok && col0 + 32 < N) store_row32<OUT, SPLIT>(y, row, col0 + 32, N, r1, sa, w_scale, sp);
             }
             tc_fence_before();
             __syncwarp();
@@ -556,13 +607,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 // (one counter per 32-row quarter of the tile) counts k-blocks merged so far;
 // the warp that brings it to num_kb writes those rows of Y and leaves ws_acc /
 // tile_count zero again.
-template <int OUT>
+template <int OUT, bool SPLIT>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                    const float* __restrict__ x_scale, const float* __restrict__ w_scale,
                    void* __restrict__ y, int M, int N, int K,
                    int32_t* __restrict__ ws_acc, unsigned int* __restrict__ tile_count,
-                   long long wait_limit) {
+                   const SplitTerm sp, long long wait_limit) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -734,7 +785,8 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                             if (OUT == kOutI32) {
                                 static_cast<int32_t*>(y)[o] = a[t];
                             } else {
-                                const float v = dequant(a[t], sa[t], sw);
+                                float v = dequant(a[t], sa[t], sw);
+                                if (SPLIT) v = add_split1(v, t, n, sp);
                                 if (OUT == kOutF32) static_cast<float*>(y)[o] = v;
                                 else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
                             }
@@ -807,27 +859,27 @@ sq_status ensure_smem_attr(Kern k, size_t bytes, bool& done) {
     return SQ_OK;
 }
 
-template <int OUT>
+template <int OUT, bool SPLIT = false>
 sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
-                       int M, int N, int K, cudaStream_t st) {
+                       int M, int N, int K, cudaStream_t st, const SplitTerm& sp = SplitTerm{}) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const size_t smem = tiled_smem_bytes();
-    sq_status r = ensure_smem_attr(gemm_tiled_kernel<OUT>, smem, attr_done[di.device & 63]);
+    sq_status r = ensure_smem_attr(gemm_tiled_kernel<OUT, SPLIT>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = tiles < di.sm_count ? tiles : di.sm_count;
-    gemm_tiled_kernel<OUT><<<grid, GEMM_THREADS, smem, st>>>(ta, tb, xs, wsc, y, M, N, K, wait_limit_cycles());
+    gemm_tiled_kernel<OUT, SPLIT><<<grid, GEMM_THREADS, smem, st>>>(ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
     return check_launch("gemm_tiled_kernel");
 }
 
-template <int OUT>
+template <int OUT, bool SPLIT = false>
 sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
-                      int M, int N, int K, cudaStream_t st) {
+                      int M, int N, int K, cudaStream_t st, const SplitTerm& sp = SplitTerm{}) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const size_t smem = pair_smem_bytes();
-    sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT>, smem, attr_done[di.device & 63]);
+    sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT, SPLIT>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const int tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int max_pairs = di.sm_count / 2;
@@ -844,23 +896,25 @@ sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float*
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<OUT>, ta, tb, xs, wsc, y, M, N, K, wait_limit_cycles());
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<OUT, SPLIT>, ta, tb, xs, wsc, y, M, N, K, sp,
+                                       wait_limit_cycles());
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(gemm_pair_kernel)");
     return check_launch("gemm_pair_kernel");
 }
 
-template <int OUT>
+template <int OUT, bool SPLIT = false>
 sq_status launch_stream(const CUtensorMap& tw, const CUtensorMap& tx, const float* xs, const float* wsc, void* y,
-                        int M, int N, int K, int32_t* ws_acc, unsigned int* counts, cudaStream_t st) {
+                        int M, int N, int K, int32_t* ws_acc, unsigned int* counts, cudaStream_t st,
+                        const SplitTerm& sp = SplitTerm{}) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const size_t smem = stream_smem_bytes();
-    sq_status r = ensure_smem_attr(gemm_stream_kernel<OUT>, smem, attr_done[di.device & 63]);
+    sq_status r = ensure_smem_attr(gemm_stream_kernel<OUT, SPLIT>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const long long units = (long long)((N + S_BM - 1) / S_BM) * ((K + BK - 1) / BK);
     const int grid = units < di.sm_count ? (int)units : di.sm_count;
-    gemm_stream_kernel<OUT><<<grid, GEMM_THREADS, smem, st>>>(tw, tx, xs, wsc, y, M, N, K, ws_acc, counts,
-                                                              wait_limit_cycles());
+    gemm_stream_kernel<OUT, SPLIT><<<grid, GEMM_THREADS, smem, st>>>(tw, tx, xs, wsc, y, M, N, K, ws_acc, counts,
+                                                                     sp, wait_limit_cycles());
     return check_launch("gemm_stream_kernel");
 }
 
@@ -881,7 +935,7 @@ size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 
 sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq, const float* w_scale,
                         int64_t M, int64_t N, int64_t K, void* y, sq_dtype out_dt, void* workspace,
-                        size_t ws_bytes, cudaStream_t st) {
+                        size_t ws_bytes, cudaStream_t st, const SplitTerm* split) {
     if (M < 0 || N < 0 || K < 0) { set_error("negative size"); return SQ_ERR_INVALID_ARG; }
     if (out_dt != SQ_F32 && out_dt != SQ_BF16 && out_dt != SQ_I32) {
         set_error("output dtype must be SQ_F32, SQ_BF16 or SQ_I32");
@@ -899,6 +953,8 @@ sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq
     }
     const int out = out_dt == SQ_F32 ? kOutF32 : (out_dt == SQ_BF16 ? kOutBF16 : kOutI32);
     sq_status r;
+    const bool sp_on = split != nullptr && split->ld > 0;
+    const SplitTerm sp = sp_on ? *split : SplitTerm{};
     if (M <= STREAM_MAX_M) {
         const size_t need = stream_ws_bytes(M, N);
         if (!workspace || ws_bytes < need) {
@@ -915,6 +971,10 @@ sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq
         int32_t* ws_acc = static_cast<int32_t*>(workspace);
         const size_t acc_al = (((size_t)M * N * 4) + 255) & ~size_t(255);
         unsigned int* counts = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + acc_al);
+        if (sp_on)
+            return out == kOutF32
+                ? launch_stream<kOutF32, true>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, ws_acc, counts, st, sp)
+                : launch_stream<kOutBF16, true>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, ws_acc, counts, st, sp);
         switch (out) {
             case kOutF32: return launch_stream<kOutF32>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, ws_acc, counts, st);
             case kOutBF16: return launch_stream<kOutBF16>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, ws_acc, counts, st);
@@ -926,6 +986,10 @@ sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq
         // paired SMs: each CTA loads 128-row boxes of A and of B
         if ((r = make_map_i8(&ta, xq, M, K, 128)) != SQ_OK) return r;
         if ((r = make_map_i8(&tb, wq, N, K, 128)) != SQ_OK) return r;
+        if (sp_on)
+            return out == kOutF32
+                ? launch_pair<kOutF32, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, sp)
+                : launch_pair<kOutBF16, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, sp);
         switch (out) {
             case kOutF32: return launch_pair<kOutF32>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
             case kOutBF16: return launch_pair<kOutBF16>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
@@ -934,11 +998,40 @@ sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq
     }
     if ((r = make_map_i8(&ta, xq, M, K, BM)) != SQ_OK) return r;
     if ((r = make_map_i8(&tb, wq, N, K, BN)) != SQ_OK) return r;
+    if (sp_on)
+        return out == kOutF32
+            ? launch_tiled<kOutF32, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, sp)
+            : launch_tiled<kOutBF16, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, sp);
     switch (out) {
         case kOutF32: return launch_tiled<kOutF32>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
         case kOutBF16: return launch_tiled<kOutBF16>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
         default: return launch_tiled<kOutI32>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st);
     }
+}
+
+sq_status gemm_split_impl(const int8_t* xq, const float* x_scale, const int8_t* wq, const float* w_scale,
+                          int64_t M, int64_t N, int64_t K, const float* x_out, const float* w_out, int64_t ld,
+                          void* y, sq_dtype out_dt, void* workspace, size_t ws_bytes, cudaStream_t st) {
+    if (out_dt != SQ_F32 && out_dt != SQ_BF16) {
+        set_error("the decomposed GEMM writes SQ_F32 or SQ_BF16 outputs");
+        return SQ_ERR_UNSUPPORTED;
+    }
+    if (ld < 0 || ld % 4 != 0 || ld > kMaxSplitLd) {
+        set_error("ld=%lld must be a multiple of 4 in [0, %d]", (long long)ld, kMaxSplitLd);
+        return SQ_ERR_UNSUPPORTED;
+    }
+    if (ld > 0 && M > 0 && N > 0) {
+        if (!x_out || !w_out) { set_error("NULL outlier operand"); return SQ_ERR_INVALID_ARG; }
+        if (!aligned16(x_out) || !aligned16(w_out)) {
+            set_error("x_out and w_out must be 16-byte aligned");
+            return SQ_ERR_UNSUPPORTED;
+        }
+    }
+    SplitTerm sp;
+    sp.x_out = x_out;
+    sp.w_out = w_out;
+    sp.ld = (int)ld;
+    return gemm_dispatch(xq, x_scale, wq, w_scale, M, N, K, y, out_dt, workspace, ws_bytes, st, &sp);
 }
 
 }  // namespace sq
@@ -953,7 +1046,15 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* x_scale, const int8_t* wq,
                        int64_t M, int64_t N, int64_t K, void* y, sq_dtype out_dt, void* workspace,
                        size_t ws_bytes, sq_stream_t stream) {
     return sq::gemm_dispatch(xq, x_scale, wq, w_scale, M, N, K, y, out_dt, workspace, ws_bytes,
-                             (cudaStream_t)stream);
+                             (cudaStream_t)stream, nullptr);
+}
+
+sq_status sq_w8a8_gemm_split(const int8_t* xq, const float* x_scale, const int8_t* wq, const float* w_scale,
+                             int64_t M, int64_t N, int64_t K, const float* x_out, const float* w_out,
+                             int64_t ld, void* y, sq_dtype out_dt, void* workspace, size_t ws_bytes,
+                             sq_stream_t stream) {
+    return sq::gemm_split_impl(xq, x_scale, wq, w_scale, M, N, K, x_out, w_out, ld, y, out_dt, workspace,
+                               ws_bytes, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -52,8 +52,10 @@ enum Site : unsigned int {
 };
 
 // Internal entry points used by sq_linear.
+struct SplitTerm;
 sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq,
                         const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
-                        sq_dtype out_dt, void* workspace, size_t ws_bytes, cudaStream_t stream);
+                        sq_dtype out_dt, void* workspace, size_t ws_bytes, cudaStream_t stream,
+                        const SplitTerm* split = nullptr);
 
 }  // namespace sq

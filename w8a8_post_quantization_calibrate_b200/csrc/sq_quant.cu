@@ -3,6 +3,7 @@
 //   a2  smoothing factors                        (sq_smooth_factors)
 //   a3  weight fold + per-output-channel int8    (sq_fold_quant_weights)
 //   a4  activation smoothing + per-token int8    (sq_smooth_quant_act)
+//   RMSNorm with the folded gain + per-token int8 (sq_rmsnorm_quant_act)
 //
 // Exactness. Every value that decides an int8 code is one correctly rounded
 // fp32 operation in the order the method defines it (explicit __fmul_rn /
@@ -50,10 +51,14 @@ struct Vec16<__nv_bfloat16> {
 constexpr int kAbsmaxThreads = 256;
 constexpr int kAbsmaxRowsInFlight = 8;   // per warp; a block covers 64 rows per iteration
 
-template <typename T>
+// TENSOR = true: the per-tensor variant. Each column maximum is first divided
+// by s_j (RN(max|x| / s_j) = max |RN(x / s_j)| for s_j > 0, because rounding
+// is monotone), the block's columns are reduced to one value, and that value
+// is merged into absmax[0].
+template <typename T, bool TENSOR>
 __global__ void __launch_bounds__(kAbsmaxThreads)
 col_absmax_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t cols,
-                  int64_t rows_per_chunk, float* __restrict__ absmax) {
+                  int64_t rows_per_chunk, float* __restrict__ absmax, const float* __restrict__ s) {
     constexpr int VEC = Vec16<T>::N;
     constexpr int TILE = 32 * VEC;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -85,12 +90,29 @@ col_absmax_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t cols,
 #pragma unroll
     for (int i = 0; i < VEC; ++i) red[warp][lane * VEC + i] = m[i];
     __syncthreads();
+    float bm = 0.0f;
     for (int c = threadIdx.x; c < TILE; c += kAbsmaxThreads) {
         float v = red[0][c];
 #pragma unroll
         for (int w = 1; w < 8; ++w) v = fmaxf(v, red[w][c]);
         const int64_t gc = (int64_t)blockIdx.x * TILE + c;
-        if (gc < cols) atomicMax(reinterpret_cast<int*>(absmax + gc), __float_as_int(v));
+        if (gc < cols) {
+            if (TENSOR) bm = fmaxf(bm, s ? __fdiv_rn(v, s[gc]) : v);
+            else atomicMax(reinterpret_cast<int*>(absmax + gc), __float_as_int(v));
+        }
+    }
+    if (TENSOR) {
+        __shared__ float bred[8];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        if (lane == 0) bred[warp] = bm;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float v = bred[0];
+#pragma unroll
+            for (int w = 1; w < 8; ++w) v = fmaxf(v, bred[w]);
+            atomicMax(reinterpret_cast<int*>(absmax), __float_as_int(v));
+        }
     }
 }
 
@@ -125,7 +147,7 @@ __global__ void smooth_factors_kernel(const float* __restrict__ xmax, const floa
 //   pass 1: v = in * s (fold, a3) or in / s (smooth, a4); running max |v|
 //   block-wide max -> scale = amax / 127 (1 for an all-zero row)
 //   pass 2: code = clamp(round_half_even(v / scale), -127, 127), 8 codes per store.
-enum RowMode { kFold = 0, kSmooth = 1 };
+enum RowMode { kFold = 0, kSmooth = 1, kNorm = 2 };
 
 template <typename T>
 struct Chunk8;
@@ -248,6 +270,14 @@ row_quant_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float*
 // The error bounds are relative and need normal numbers: a row whose
 // approximate maximum is below 2^-90 (this includes all-zero rows) is
 // quantized entirely with exact divisions.
+//
+// kNorm (RMSNorm with the smoothing folded into its gain, m_j = g'_j): the
+// row's factor r = RN32(1 / sqrt(sum x^2 / K + eps)) comes first, the sum of
+// squares in fp64 (every square exact) reduced over the group, then
+// 1/sqrt in correctly rounded fp64 operations. The norm output
+// v_j = RN(RN(x_j * r) * g'_j) is an exact product chain, so the candidates
+// and codes follow the fold argument with r as a common positive factor
+// (pass 2 forms q' = RN(v_j * RN(1/scale)), within 4 ulp of q*).
 constexpr float kMagic = 12582912.0f;            // 1.5 * 2^23
 constexpr float kTieGuard = 1.0f / 8192.0f;      // >> 5.3e-5, the bound on |q' - q*|
 constexpr float kCandidate = 1.0f - 1.0f / 64.0f;
@@ -341,8 +371,15 @@ struct RawChunk<float> {
 // scale)), -127, 127) with v = RN(x * s_j) (fold) or RN(x / s_j) (smooth).
 // Out of line: these run only on the rare near-tie and small-row paths.
 template <int MODE>
-__device__ __noinline__ uint32_t exact_code(float x, float s_j, float scale) {
-    const float v = MODE == kFold ? __fmul_rn(x, s_j) : __fdiv_rn(x, s_j);
+__device__ __forceinline__ float exact_value(float x, float m_j, float r) {
+    if (MODE == kFold) return __fmul_rn(x, m_j);
+    if (MODE == kSmooth) return __fdiv_rn(x, m_j);
+    return __fmul_rn(__fmul_rn(x, r), m_j);
+}
+
+template <int MODE>
+__device__ __noinline__ uint32_t exact_code(float x, float s_j, float scale, float r) {
+    const float v = exact_value<MODE>(x, s_j, r);
     int qi = __float2int_rn(__fdiv_rn(v, scale));
     qi = max(-127, min(127, qi));
     return (uint32_t)qi & 0xffu;
@@ -350,8 +387,23 @@ __device__ __noinline__ uint32_t exact_code(float x, float s_j, float scale) {
 
 // |v| of one element, exactly (v as above).
 template <int MODE>
-__device__ __noinline__ float exact_abs(float x, float s_j) {
-    return fabsf(MODE == kFold ? __fmul_rn(x, s_j) : __fdiv_rn(x, s_j));
+__device__ __noinline__ float exact_abs(float x, float s_j, float r) {
+    return fabsf(exact_value<MODE>(x, s_j, r));
+}
+
+// Sum over the R warps of a group, in fp64 (same slot scheme as group_max).
+template <int R>
+__device__ __forceinline__ double group_sum(double v, double* red, int grp, int wig, int lane, int bank) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (R == 1) return v;
+    double* slot = red + (grp * 2 + bank) * R;
+    if (lane == 0) slot[wig] = v;
+    asm volatile("bar.sync %0, %1;" :: "r"(1 + grp), "r"(32 * R) : "memory");
+    v = slot[0];
+#pragma unroll
+    for (int w = 1; w < R; ++w) v += slot[w];
+    return v;
 }
 
 template <int R>
@@ -374,7 +426,8 @@ constexpr int row_fast_threads() { return 32 * R > 256 ? 32 * R : 256; }
 template <typename T, int MODE, int R, int CPL>
 __global__ void __launch_bounds__(row_fast_threads<R>(), R >= 16 ? 1 : (R >= 8 ? 2 : 4))
 row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
-                      int8_t* __restrict__ q, float* __restrict__ scale_out) {
+                      int8_t* __restrict__ q, float* __restrict__ scale_out, float eps,
+                      float* __restrict__ r_out) {
     extern __shared__ float smem[];
     const int64_t nchunks = K >> 3;
     float* mul_lo = smem;                                                // [nchunks][4] fp32, elements 0..3
@@ -383,6 +436,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
     float* red = smem + nchunks * 12;                                    // [groups][2][R]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int groups = blockDim.x / (32 * R);
+    double* red64 = reinterpret_cast<double*>(red + groups * 2 * R);     // [groups][2][R] (kNorm)
     const int grp = warp / R, wig = warp % R;
     const int gl = wig * 32 + lane;          // lane index inside the group
 
@@ -401,7 +455,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
     __syncthreads();
 
     const uint64_t mag2 = f2_pack(kMagic, kMagic);
-    int bank = 0;
+    int bank = 0, bank64 = 0;
     // Long rows (R >= 8) double-buffer the row in registers: the next row's
     // loads are issued before the current row is processed.
     constexpr bool kPrefetch = R >= 8;
@@ -438,6 +492,27 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
             }
         }
 
+        // ---- RMSNorm factor of the row
+        float rn = 1.0f;
+        if (MODE == kNorm) {
+            double ss = 0.0;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int64_t c = gl + (int64_t)i * 32 * R;
+                if (c < nchunks) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const double v = (double)raw[i].get(e);
+                        ss = __fma_rn(v, v, ss);
+                    }
+                }
+            }
+            ss = group_sum<R>(ss, red64, grp, wig, lane, bank64);
+            bank64 ^= 1;
+            rn = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)eps))));
+            if (r_out != nullptr && gl == 0) r_out[row] = rn;
+        }
+
         // ---- pass 1: approximate chunk maxima
         float cm[CPL];
         float m = 0.0f;
@@ -462,7 +537,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
         bank ^= 1;
         int8_t* rq = q + row * K;
 
-        if (!(mrow >= kSmallRow)) {
+        if (!((MODE == kNorm ? __fmul_rn(mrow, rn) : mrow) >= kSmallRow)) {
             // zero, tiny or near-underflow row: exact maximum and codes
             float ex = 0.0f;
 #pragma unroll
@@ -470,7 +545,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
                 const int64_t c = gl + (int64_t)i * 32 * R;
                 if (c < nchunks)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(raw[i].get(e), __ldg(s + c * 8 + e)));
+                    for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), rn));
             }
             const float a = group_max<R>(ex, red, grp, wig, lane, bank);
             bank ^= 1;
@@ -482,7 +557,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
                     uint32_t b[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        b[e] = a == 0.0f ? 0u : exact_code<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), scale);
+                        b[e] = a == 0.0f ? 0u : exact_code<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), scale, rn);
                     *reinterpret_cast<uint2*>(rq + c * 8) =
                         make_uint2(b[0] | b[1] << 8 | b[2] << 16 | b[3] << 24, b[4] | b[5] << 8 | b[6] << 16 | b[7] << 24);
                 }
@@ -499,7 +574,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
             if (cm[i] >= tau) {
                 const int64_t c = gl + (int64_t)i * 32 * R;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(raw[i].get(e), __ldg(s + c * 8 + e)));
+                for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), rn));
             }
         }
         const float amax = group_max<R>(ex, red, grp, wig, lane, bank);
@@ -509,6 +584,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
         const float scale = __fdiv_rn(amax, 127.0f);
         const float r = __frcp_rn(scale);
         const uint64_t r2 = f2_pack(r, r);
+        const uint64_t rn2 = f2_pack(rn, rn);
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
             const int64_t c = gl + (int64_t)i * 32 * R;
@@ -520,7 +596,8 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
                 bool near_tie = false;
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const uint64_t q2 = f2_mul(f2_mul(raw[i].pair(p), mp[p]), r2);
+                    const uint64_t x2 = MODE == kNorm ? f2_mul(raw[i].pair(p), rn2) : raw[i].pair(p);
+                    const uint64_t q2 = f2_mul(f2_mul(x2, mp[p]), r2);
                     const uint64_t t2 = f2_add(q2, mag2);
                     const uint64_t d2 = f2_sub(q2, f2_sub(t2, mag2));
                     float t0, t1, d0, d1;
@@ -535,9 +612,10 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
                     const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float qv = __fmul_rn(__fmul_rn(raw[i].get(e), mv[e]), r);
+                        const float xe = MODE == kNorm ? __fmul_rn(raw[i].get(e), rn) : raw[i].get(e);
+                        const float qv = __fmul_rn(__fmul_rn(xe, mv[e]), r);
                         const float d = __fsub_rn(qv, __fsub_rn(__fadd_rn(qv, kMagic), kMagic));
-                        if (fabsf(d) >= 0.5f - kTieGuard) t[e] = exact_code<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), scale);
+                        if (fabsf(d) >= 0.5f - kTieGuard) t[e] = exact_code<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), scale, rn);
                     }
                 }
                 const uint32_t lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
@@ -583,13 +661,13 @@ int pow2ceil(int64_t v) {
 
 template <typename T, int MODE, int R>
 sq_status launch_row_quant_fast_inst(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
-                                     float* scale, cudaStream_t st) {
+                                     float* scale, cudaStream_t st, float eps, float* r_out) {
     constexpr int CPL = RowFastCPL<T>::value;
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const int threads = 32 * R > 256 ? 32 * R : 256;
     const int groups = threads / (32 * R);
-    const size_t smem = (size_t)K * 6 + (size_t)groups * 2 * R * sizeof(float);
+    const size_t smem = (size_t)K * 6 + (size_t)groups * 2 * R * (sizeof(float) + (MODE == kNorm ? sizeof(double) : 0));
     auto kern = row_quant_fast_kernel<T, MODE, R, CPL>;
     if (!attr_done[di.device & 63]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -604,13 +682,13 @@ sq_status launch_row_quant_fast_inst(const void* in, int64_t rows, int64_t K, co
     const int64_t need = (rows + groups - 1) / groups;
     const int64_t max_blocks = (int64_t)di.sm_count * per_sm;
     const int grid = (int)(need < max_blocks ? need : max_blocks);
-    kern<<<grid, threads, smem, st>>>(static_cast<const T*>(in), rows, K, s, q, scale);
+    kern<<<grid, threads, smem, st>>>(static_cast<const T*>(in), rows, K, s, q, scale, eps, r_out);
     return check_launch("row_quant_fast_kernel");
 }
 
 template <typename T, int MODE>
 sq_status launch_row_quant(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
-                           float* scale, cudaStream_t st) {
+                           float* scale, cudaStream_t st, float eps = 0.0f, float* r_out = nullptr) {
     constexpr int CPL = RowFastCPL<T>::value;
     const int64_t nchunks = K / 8;
     // the fewest warps per row whose lanes hold the row in CPL chunks each
@@ -618,15 +696,20 @@ sq_status launch_row_quant(const void* in, int64_t rows, int64_t K, const float*
         for (int R = 1; R <= 16; R *= 2) {
             if (nchunks <= (int64_t)32 * R * CPL) {
                 switch (R) {
-                    case 1: return launch_row_quant_fast_inst<T, MODE, 1>(in, rows, K, s, q, scale, st);
-                    case 2: return launch_row_quant_fast_inst<T, MODE, 2>(in, rows, K, s, q, scale, st);
-                    case 4: return launch_row_quant_fast_inst<T, MODE, 4>(in, rows, K, s, q, scale, st);
-                    case 8: return launch_row_quant_fast_inst<T, MODE, 8>(in, rows, K, s, q, scale, st);
-                    default: return launch_row_quant_fast_inst<T, MODE, 16>(in, rows, K, s, q, scale, st);
+                    case 1: return launch_row_quant_fast_inst<T, MODE, 1>(in, rows, K, s, q, scale, st, eps, r_out);
+                    case 2: return launch_row_quant_fast_inst<T, MODE, 2>(in, rows, K, s, q, scale, st, eps, r_out);
+                    case 4: return launch_row_quant_fast_inst<T, MODE, 4>(in, rows, K, s, q, scale, st, eps, r_out);
+                    case 8: return launch_row_quant_fast_inst<T, MODE, 8>(in, rows, K, s, q, scale, st, eps, r_out);
+                    default: return launch_row_quant_fast_inst<T, MODE, 16>(in, rows, K, s, q, scale, st, eps, r_out);
                 }
             }
         }
     }
+    if constexpr (MODE == kNorm) {
+        set_error("K=%lld exceeds the fused norm-and-quantize limit of %lld for this dtype", (long long)K,
+                  (long long)(32 * 16 * 8 * RowFastCPL<T>::value));
+        return SQ_ERR_UNSUPPORTED;
+    } else {
     // longer rows: the IEEE-division kernel
     int64_t tpb = pow2ceil((nchunks + 3) / 4);
     if (tpb < 128) tpb = 128;
@@ -642,6 +725,7 @@ sq_status launch_row_quant(const void* in, int64_t rows, int64_t K, const float*
         case 256: return launch_row_quant_tpb<T, MODE, 256>(maxc, in, rows, K, s, q, scale, st);
         case 512: return launch_row_quant_tpb<T, MODE, 512>(maxc, in, rows, K, s, q, scale, st);
         default: return launch_row_quant_tpb<T, MODE, 1024>(maxc, in, rows, K, s, q, scale, st);
+    }
     }
 }
 
@@ -675,23 +759,17 @@ sq_status check_matrix(const void* p, int64_t rows, int64_t cols, const char* na
 
 }  // namespace
 
-sq_status calibrate_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_t cols,
-                                float* absmax, cudaStream_t st) {
-    sq_status r;
-    if ((r = check_input_dtype(dt)) != SQ_OK) return r;
-    if ((r = check_matrix(x, rows, cols, "x")) != SQ_OK) return r;
-    if (cols > 0 && !absmax) { set_error("absmax: NULL pointer"); return SQ_ERR_INVALID_ARG; }
-    if (rows == 0 || cols == 0) return SQ_OK;
-    const int es = dt == SQ_F32 ? 4 : 2;
+// About one wave of 256-thread blocks (8 per SM); every block covers a
+// multiple of the 64 rows it reads per iteration. Returns the grid and the rows
+// per block.
+sq_status absmax_grid(int64_t rows, int64_t cols, int es, dim3& grid, int64_t& per) {
     const int64_t tile = 32 * (16 / es);
     const int64_t ct = (cols + tile - 1) / tile;
-    // About one wave of 256-thread blocks (8 per SM); every block covers a
-    // multiple of the 64 rows it reads per iteration.
     const int64_t step_rows = 8 * kAbsmaxRowsInFlight;
     const int64_t target = (int64_t)device_info().sm_count * 8;
     int64_t rc = target / ct;
     if (rc < 1) rc = 1;
-    int64_t per = (rows + rc - 1) / rc;
+    per = (rows + rc - 1) / rc;
     per = (per + step_rows - 1) / step_rows * step_rows;
     rc = (rows + per - 1) / per;
     if (rc > 65535) {
@@ -701,13 +779,26 @@ sq_status calibrate_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_
         rc = (rows + per - 1) / per;
     }
     if (ct > 2147483647LL) { set_error("cols too large"); return SQ_ERR_UNSUPPORTED; }
-    dim3 grid((unsigned)ct, (unsigned)rc);
+    grid = dim3((unsigned)ct, (unsigned)rc);
+    return SQ_OK;
+}
+
+sq_status calibrate_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_t cols,
+                                float* absmax, cudaStream_t st) {
+    sq_status r;
+    if ((r = check_input_dtype(dt)) != SQ_OK) return r;
+    if ((r = check_matrix(x, rows, cols, "x")) != SQ_OK) return r;
+    if (cols > 0 && !absmax) { set_error("absmax: NULL pointer"); return SQ_ERR_INVALID_ARG; }
+    if (rows == 0 || cols == 0) return SQ_OK;
+    dim3 grid;
+    int64_t per = 0;
+    if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
     if (dt == SQ_F32)
-        col_absmax_kernel<float><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, absmax);
+        col_absmax_kernel<float, false><<<grid, kAbsmaxThreads, 0, st>>>(
+            static_cast<const uint8_t*>(x), rows, cols, per, absmax, nullptr);
     else
-        col_absmax_kernel<__nv_bfloat16><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, absmax);
+        col_absmax_kernel<__nv_bfloat16, false><<<grid, kAbsmaxThreads, 0, st>>>(
+            static_cast<const uint8_t*>(x), rows, cols, per, absmax, nullptr);
     return check_launch("col_absmax_kernel");
 }
 

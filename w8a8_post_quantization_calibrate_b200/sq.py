@@ -43,6 +43,17 @@ _SIGS = {
     "sq_smooth_factors": ([_vp, _vp, _i64, _f32, _f32, _vp, _vp], _int),
     "sq_fold_quant_weights": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_smooth_quant_act": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "sq_tensor_absmax": ([_vp, _int, _i64, _i64, _vp, _vp, _vp], _int),
+    "sq_quant_act_per_tensor": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp], _int),
+    "sq_fold_norm_gain": ([_vp, _int, _i64, _vp, _vp, _vp], _int),
+    "sq_rmsnorm_quant_act": ([_vp, _int, _i64, _i64, _vp, _f32, _vp, _vp, _vp, _vp], _int),
+    "sq_outlier_split": ([_vp, _i64, _f32, _vp, _vp, _vp, _vp], _int),
+    "sq_quant_bulk": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "sq_gather_columns": ([_vp, _int, _i64, _i64, _vp, _i64, _i64, _vp, _vp], _int),
+    "sq_w8a8_gemm_split": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _int, _vp, _sz, _vp],
+                           _int),
+    "sq_alpha_search_workspace_size": ([_i64, _i64, _i64, _i64], _sz),
+    "sq_alpha_search": ([_vp, _vp, _int, _i64, _i64, _i64, _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp], _int),
     "sq_w8a8_gemm_workspace_size": ([_i64, _i64, _i64], _sz),
     "sq_w8a8_gemm": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp], _int),
     "sq_w8a8_gemm_noalloc": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp], _int),
@@ -150,6 +161,63 @@ def sq_smooth_quant_act(x: torch.Tensor, s: torch.Tensor, xq: torch.Tensor | Non
     return xq, x_scale
 
 
+def _opt_dev(t: torch.Tensor | None, name: str):
+    return None if t is None else _dev(t, name)
+
+
+def sq_tensor_absmax(x: torch.Tensor, s: torch.Tensor | None, amax: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Running per-tensor max |x / s_j| into `amax` (float32 [1], in/out; a
+    fresh zero tensor if not given). s None: max |x|."""
+    rows, cols = x.shape
+    if amax is None:
+        amax = torch.zeros(1, dtype=torch.float32, device=x.device)
+    _check(_lib.sq_tensor_absmax(_dev(x, "x"), _dt(x), rows, cols, _opt_dev(s, "s"), _dev(amax, "amax"),
+                                 _stream(stream)), "sq_tensor_absmax")
+    return amax
+
+
+def sq_quant_act_per_tensor(x: torch.Tensor, s: torch.Tensor | None, amax: torch.Tensor,
+                            xq: torch.Tensor | None = None, x_scale: torch.Tensor | None = None,
+                            stream=None):
+    T, K = x.shape
+    if xq is None:
+        xq = torch.empty((T, K), dtype=torch.int8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(_lib.sq_quant_act_per_tensor(_dev(x, "x"), _dt(x), T, K, _opt_dev(s, "s"), _dev(amax, "amax"),
+                                        _dev(xq, "xq"), _dev(x_scale, "x_scale"), _stream(stream)),
+           "sq_quant_act_per_tensor")
+    return xq, x_scale
+
+
+def sq_fold_norm_gain(gain: torch.Tensor, s: torch.Tensor, gain_folded: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    K = gain.shape[0]
+    if gain_folded is None:
+        gain_folded = torch.empty(K, dtype=torch.float32, device=gain.device)
+    _check(_lib.sq_fold_norm_gain(_dev(gain, "gain"), _dt(gain), K, _dev(s, "s"),
+                                  _dev(gain_folded, "gain_folded"), _stream(stream)), "sq_fold_norm_gain")
+    return gain_folded
+
+
+def sq_rmsnorm_quant_act(x: torch.Tensor, gain_folded: torch.Tensor, eps: float,
+                         xq: torch.Tensor | None = None, x_scale: torch.Tensor | None = None,
+                         inv_rms: torch.Tensor | None = None, want_inv_rms: bool = True, stream=None):
+    """RMSNorm with the folded gain, then per-token int8 -> (xq, x_scale, inv_rms or None)."""
+    T, K = x.shape
+    if xq is None:
+        xq = torch.empty((T, K), dtype=torch.int8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(T, dtype=torch.float32, device=x.device)
+    if inv_rms is None and want_inv_rms:
+        inv_rms = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(_lib.sq_rmsnorm_quant_act(_dev(x, "x"), _dt(x), T, K, _dev(gain_folded, "gain_folded"),
+                                     float(eps), _dev(xq, "xq"), _dev(x_scale, "x_scale"),
+                                     _opt_dev(inv_rms, "inv_rms"), _stream(stream)), "sq_rmsnorm_quant_act")
+    return xq, x_scale, inv_rms
+
+
 def sq_w8a8_gemm_workspace_size(M: int, N: int, K: int) -> int:
     return int(_lib.sq_w8a8_gemm_workspace_size(M, N, K))
 
@@ -205,6 +273,83 @@ def sq_w8a8_gemm_noalloc(xq: torch.Tensor, x_scale: torch.Tensor | None, wq: tor
                                      M, N, K, _dev(y, "y"), _dt(y), _stream(stream)),
            "sq_w8a8_gemm_noalloc")
     return y
+
+
+def sq_outlier_split(xmax: torch.Tensor, threshold: float, stream=None):
+    """-> (keep float32 [K], idx int32 [K] (first `count` valid), count int32 [1]), all on the device."""
+    K = xmax.shape[0]
+    keep = torch.empty(K, dtype=torch.float32, device=xmax.device)
+    idx = torch.empty(max(K, 1), dtype=torch.int32, device=xmax.device)
+    count = torch.empty(1, dtype=torch.int32, device=xmax.device)
+    _check(_lib.sq_outlier_split(_dev(xmax, "xmax"), K, float(threshold), _dev(keep, "keep"), _dev(idx, "idx"),
+                                 _dev(count, "count"), _stream(stream)), "sq_outlier_split")
+    return keep, idx, count
+
+
+def sq_quant_bulk(x: torch.Tensor, keep: torch.Tensor, q: torch.Tensor | None = None,
+                  scale: torch.Tensor | None = None, stream=None):
+    rows, K = x.shape
+    if q is None:
+        q = torch.empty((rows, K), dtype=torch.int8, device=x.device)
+    if scale is None:
+        scale = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(_lib.sq_quant_bulk(_dev(x, "x"), _dt(x), rows, K, _dev(keep, "keep"), _dev(q, "q"),
+                              _dev(scale, "scale"), _stream(stream)), "sq_quant_bulk")
+    return q, scale
+
+
+def sq_gather_columns(x: torch.Tensor, idx: torch.Tensor, n: int, ld: int, out: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    rows, K = x.shape
+    if out is None:
+        out = torch.empty((rows, ld), dtype=torch.float32, device=x.device)
+    _check(_lib.sq_gather_columns(_dev(x, "x"), _dt(x), rows, K, _dev(idx, "idx"), int(n), int(ld),
+                                  _dev(out, "out"), _stream(stream)), "sq_gather_columns")
+    return out
+
+
+def sq_w8a8_gemm_split(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                       x_out: torch.Tensor, w_out: torch.Tensor, out_dtype=torch.bfloat16,
+                       y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    M, K = xq.shape
+    N = wq.shape[0]
+    ld = x_out.shape[1]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, xq.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.sq_w8a8_gemm_split(_dev(xq, "xq"), _dev(x_scale, "x_scale"), _dev(wq, "wq"),
+                                   _dev(w_scale, "w_scale"), M, N, K, _dev(x_out, "x_out"), _dev(w_out, "w_out"),
+                                   ld, _dev(y, "y"), _dt(y), ws_ptr, ws_bytes, _stream(stream)),
+           "sq_w8a8_gemm_split")
+    return y
+
+
+def sq_alpha_search_workspace_size(T: int, N: int, K: int, n_alpha: int) -> int:
+    return int(_lib.sq_alpha_search_workspace_size(T, N, K, n_alpha))
+
+
+def sq_alpha_search(x: torch.Tensor, w: torch.Tensor, alphas, eps: float = 1e-8,
+                    workspace: torch.Tensor | None = None, stream=None):
+    """W8A8 relative output error for each alpha on the calibration batch x
+    -> (errors list of float, best alpha). Synchronizes the stream."""
+    T, K = x.shape
+    N = w.shape[0]
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must have the same dtype")
+    a = (ctypes.c_float * len(alphas))(*[float(v) for v in alphas])
+    err = (ctypes.c_double * len(alphas))()
+    best = ctypes.c_float(0.0)
+    need = sq_alpha_search_workspace_size(T, N, K, len(alphas))
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    _check(_lib.sq_alpha_search(_dev(x, "x"), _dev(w, "w"), _dt(x), T, N, K, ctypes.cast(a, _vp), len(alphas),
+                                float(eps), ctypes.cast(err, _vp), ctypes.cast(ctypes.pointer(best), _vp),
+                                workspace.data_ptr(), workspace.numel(), _stream(stream)), "sq_alpha_search")
+    return list(err), float(best.value)
 
 
 def sq_linear_workspace_size(M: int, N: int, K: int, in_dtype=torch.bfloat16, out_dtype=torch.bfloat16) -> int:
