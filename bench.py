@@ -212,6 +212,99 @@ def workload_inputs(name: str, decode_m: int):
     return wl, x, w
 
 
+VARIANTS = {
+    "smoothquant": "a1(X) a1(W) a2 a3 a4 a5: per-token dynamic activation scales (O1)",
+    "per_tensor_dynamic": "a1(X) a1(W) a2 a3, per-tensor range of X/s, per-tensor codes, a5 (O2)",
+    "per_tensor_static": "a1(X) a1(W) a2 a3, static range from the calibration maxima, per-tensor codes, a5 (O3)",
+    "rmsnorm": "a1(X) a1(W) a2 a3, gain fold, RMSNorm + per-token codes, a5 (the norm-folded O1)",
+    "split": "a1(X), outlier split, bulk int8 of W and X, outlier gathers, int8 GEMM + fp32 outlier epilogue",
+}
+SPLIT_THRESHOLD = 6.0  # outlier channels: calibration maximum >= 6 (the synthetic outliers are 20-80x)
+
+
+def build_step(variant, sq, wl, x, w, dev, stream):
+    """Buffers and the ordered stages of one step: [(name, callable, algorithmic
+    bytes, ops)]. Every callable is one C ABI call on `stream`."""
+    M, K = x.shape
+    N = w.shape[0]
+    in_es = x.element_size()
+    out_es = torch.empty(0, dtype=wl.out_dtype).element_size()
+    maxima = torch.zeros(2 * K + 4, dtype=torch.float32, device=dev)   # xmax | wmax | amax, cleared per step
+    xmax, wmax, amax = maxima[:K], maxima[K:2 * K], maxima[2 * K:2 * K + 1]
+    s = torch.empty(K, dtype=torch.float32, device=dev)
+    wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+    wsc = torch.empty(N, dtype=torch.float32, device=dev)
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    xsc = torch.empty(M, dtype=torch.float32, device=dev)
+    y = torch.empty((M, N), dtype=wl.out_dtype, device=dev)
+    gws = sq.gemm_workspace(M, N, K, dev)
+    ops = 2.0 * M * N * K
+    gemm_bytes = M * K + N * K + M * 4 + N * 4 + M * N * out_es
+    st = []
+    st.append(("a1_calibrate_x", lambda: sq.sq_calibrate_absmax(x, xmax, stream=stream), M * K * in_es + K * 4, 0))
+    if variant == "split":
+        keep = torch.empty(K, dtype=torch.float32, device=dev)
+        idx = torch.empty(K, dtype=torch.int32, device=dev)
+        count = torch.empty(1, dtype=torch.int32, device=dev)
+        # the outlier set is static: its size is fixed once, from this workload's calibration
+        sq.sq_calibrate_absmax(x, xmax, stream=stream)
+        _, _, c0 = sq.sq_outlier_split(xmax, SPLIT_THRESHOLD, stream=stream)
+        n_out = int(c0.item())
+        ld = max(4, (n_out + 3) // 4 * 4)
+        xo = torch.empty((M, ld), dtype=torch.float32, device=dev)
+        wo = torch.empty((N, ld), dtype=torch.float32, device=dev)
+
+        st.append(("outlier_split", lambda: sq.sq_outlier_split(xmax, SPLIT_THRESHOLD, keep=keep, idx=idx, count=count,
+                                                                stream=stream), K * 4 * 2 + K * 4, 0))
+        st.append(("quant_bulk_w", lambda: sq.sq_quant_bulk(w, keep, q=wq, scale=wsc, stream=stream),
+                   N * K * in_es + K * 4 + N * K + N * 4, 0))
+        st.append(("quant_bulk_x", lambda: sq.sq_quant_bulk(x, keep, q=xq, scale=xsc, stream=stream),
+                   M * K * in_es + K * 4 + M * K + M * 4, 0))
+        st.append(("gather_x", lambda: sq.sq_gather_columns(x, idx, n_out, ld, out=xo, stream=stream),
+                   M * n_out * in_es + M * ld * 4, 0))
+        st.append(("gather_w", lambda: sq.sq_gather_columns(w, idx, n_out, ld, out=wo, stream=stream),
+                   N * n_out * in_es + N * ld * 4, 0))
+        st.append(("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm_split(xq, xsc, wq, wsc, xo, wo, y=y, workspace=gws,
+                                                                  stream=stream),
+                   gemm_bytes + (M + N) * ld * 4, ops))
+        return maxima, st, {"outlier_channels": n_out, "ld": ld, "threshold": SPLIT_THRESHOLD}
+    st.append(("a1_calibrate_w", lambda: sq.sq_calibrate_absmax(w, wmax, stream=stream), N * K * in_es + K * 4, 0))
+    st.append(("a2_smooth_factors", lambda: sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream),
+               3 * K * 4, 0))
+    st.append(("a3_fold_quant_w", lambda: sq.sq_fold_quant_weights(w, s, wq=wq, w_scale=wsc, stream=stream),
+               N * K * in_es + K * 4 + N * K + N * 4, 0))
+    act_bytes = M * K * in_es + K * 4 + M * K + M * 4
+    extra = {}
+    if variant == "smoothquant":
+        st.append(("a4_smooth_quant_x", lambda: sq.sq_smooth_quant_act(x, s, xq=xq, x_scale=xsc, stream=stream),
+                   act_bytes, 0))
+    elif variant == "per_tensor_dynamic":
+        st.append(("tensor_absmax_x", lambda: sq.sq_tensor_absmax(x, s, amax, stream=stream),
+                   M * K * in_es + K * 4 + 4, 0))
+        st.append(("quant_per_tensor_x", lambda: sq.sq_quant_act_per_tensor(x, s, amax, xq=xq, x_scale=xsc,
+                                                                            stream=stream),
+                   act_bytes, 0))
+    elif variant == "per_tensor_static":
+        st.append(("static_range", lambda: sq.sq_tensor_absmax(xmax.view(1, K), s, amax, stream=stream),
+                   2 * K * 4 + 4, 0))
+        st.append(("quant_per_tensor_x", lambda: sq.sq_quant_act_per_tensor(x, s, amax, xq=xq, x_scale=xsc,
+                                                                            stream=stream),
+                   act_bytes, 0))
+    elif variant == "rmsnorm":
+        gain = torch.from_numpy(np.random.default_rng(0).uniform(0.5, 1.5, K).astype(np.float32)).to(dev)
+        gf = torch.empty(K, dtype=torch.float32, device=dev)
+        st.append(("fold_norm_gain", lambda: sq.sq_fold_norm_gain(gain, s, gain_folded=gf, stream=stream),
+                   3 * K * 4, 0))
+        st.append(("rmsnorm_quant_x", lambda: sq.sq_rmsnorm_quant_act(x, gf, 1e-5, xq=xq, x_scale=xsc,
+                                                                      want_inv_rms=False, stream=stream),
+                   act_bytes, 0))
+        extra = {"norm_eps": 1e-5, "note": "x plays the hidden state; s from its maxima (kernel cost is "
+                                           "independent of the values of s)"}
+    st.append(("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm(xq, xsc, wq, wsc, y=y, workspace=gws, stream=stream),
+               gemm_bytes, ops))
+    return maxima, st, extra
+
+
 def run_ours(args, world, rank, local):
     from w8a8_post_quantization_calibrate_b200 import sq
     dev = torch.device("cuda", local)
@@ -225,17 +318,9 @@ def run_ours(args, world, rank, local):
     in_es, out_es = x_cpu.element_size(), torch.empty(0, dtype=wl.out_dtype).element_size()
     stream = torch.cuda.current_stream(dev)
 
-    xmax = torch.zeros(K, dtype=torch.float32, device=dev)
-    wmax = torch.zeros(K, dtype=torch.float32, device=dev)
-    maxima = torch.cat([xmax, wmax])  # one buffer, cleared once per step
-    xmax, wmax = maxima[:K], maxima[K:]
-    s = torch.empty(K, dtype=torch.float32, device=dev)
-    wq = torch.empty((N, K), dtype=torch.int8, device=dev)
-    wsc = torch.empty(N, dtype=torch.float32, device=dev)
-    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
-    xsc = torch.empty(M, dtype=torch.float32, device=dev)
-    y = torch.empty((M, N), dtype=wl.out_dtype, device=dev)
-    gws = sq.gemm_workspace(M, N, K, dev)
+    maxima, stages, variant_info = build_step(args.variant, sq, wl, x, w, dev, stream)
+    names = [n for n, _, _, _ in stages]
+    nst = len(stages)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
@@ -245,25 +330,14 @@ def run_ours(args, world, rank, local):
         # kernel would pay for.
         flush.zero_()
         flush_read.amax()
-    names = ["a1_calibrate_x", "a1_calibrate_w", "a2_smooth_factors", "a3_fold_quant_w",
-             "a4_smooth_quant_x", "a5_w8a8_gemm"]
-    launches_per_step = len(names)
+    launches_per_step = nst
 
     def step(ev=None):
         maxima.zero_()
-        if ev: ev[0].record(stream)
-        sq.sq_calibrate_absmax(x, xmax, stream=stream)
-        if ev: ev[1].record(stream)
-        sq.sq_calibrate_absmax(w, wmax, stream=stream)
-        if ev: ev[2].record(stream)
-        sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream)
-        if ev: ev[3].record(stream)
-        sq.sq_fold_quant_weights(w, s, wq=wq, w_scale=wsc, stream=stream)
-        if ev: ev[4].record(stream)
-        sq.sq_smooth_quant_act(x, s, xq=xq, x_scale=xsc, stream=stream)
-        if ev: ev[5].record(stream)
-        sq.sq_w8a8_gemm(xq, xsc, wq, wsc, y=y, workspace=gws, stream=stream)
-        if ev: ev[6].record(stream)
+        for j, (_, fn, _, _) in enumerate(stages):
+            if ev: ev[j].record(stream)
+            fn()
+        if ev: ev[nst].record(stream)
 
     for _ in range(args.warmup):
         flush_l2()
@@ -272,7 +346,7 @@ def run_ours(args, world, rank, local):
     if sq.sq_get_status(stream) != sq.SQ_OK:
         raise RuntimeError("device status error during warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
@@ -288,7 +362,7 @@ def run_ours(args, world, rank, local):
     per_kernel = {n: 0.0 for n in names}
     step_ms = 0.0
     for ev in events:
-        step_ms += ev[0].elapsed_time(ev[6])
+        step_ms += ev[0].elapsed_time(ev[nst])
         for j, n in enumerate(names):
             per_kernel[n] += ev[j].elapsed_time(ev[j + 1])
     step_ms /= args.steps
@@ -301,7 +375,7 @@ def run_ours(args, world, rank, local):
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     int8_peak = bf16_peak * INT8_OVER_BF16
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    kb = kernel_bytes(M, N, K, in_es, out_es)
+    kb = {n: b for n, _, b, _ in stages}
     kernels = {}
     for n in names:
         ms = per_kernel[n]
@@ -313,11 +387,13 @@ def run_ours(args, world, rank, local):
         kernels[n] = entry
     gemm_ms = per_kernel["a5_w8a8_gemm"]
     achieved = ops / (gemm_ms * 1e-3) / 1e12
+    default_gemm = args.variant != "split"
     if M > 16:
         roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel (a5, paired-SM tcgen05)" if M > 128
                     else "gemm_tiled_kernel (a5)",
                     "achieved": round(achieved, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
-                    "frac": round(achieved / int8_peak, 4), "traffic": load_traffic() if M > 128 else None,
+                    "frac": round(achieved / int8_peak, 4),
+                    "traffic": load_traffic() if (M > 128 and default_gemm) else None,
                     "peak_source": f"{peak_src}: bf16 {bf16_peak} TFLOP/s (burst) x {INT8_OVER_BF16} nominal "
                                    f"int8/bf16 ratio",
                     "algorithmic_ops_per_launch": ops}
@@ -330,7 +406,7 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public API: pinned host X and W in, host Y out
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and args.variant == "smoothquant":
         xh = x_cpu.pin_memory()
         wh = w_cpu.pin_memory()
         yh = torch.empty((M, N), dtype=wl.out_dtype).pin_memory()
@@ -356,7 +432,7 @@ def run_ours(args, world, rank, local):
                "api": "sq_linear (C ABI) with pinned host buffers"}
 
     cpu_baseline = None
-    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+    if rank == 0 and world == 1 and args.cpu_seconds > 0 and args.variant == "smoothquant":
         v, cores, desc, _ = oracle_sample(x_cpu, w_cpu, wl.alpha, args.cpu_seconds)
         cpu_baseline = {"value": round(v, 5), "unit": "TOPS", "cores": cores, "kind": "oracle",
                         "sample": desc}
@@ -375,8 +451,9 @@ def run_ours(args, world, rank, local):
                    "out_dtype": str(wl.out_dtype).replace("torch.", ""),
                    "alpha": wl.alpha, "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "step": "a1(X) a1(W) a2 a3 a4 a5, one stream"},
-        "act_quant_gbs": kernels["a4_smooth_quant_x"]["gbs"],
+                   "variant": args.variant, "step": VARIANTS[args.variant] + ", one stream", **variant_info},
+        "act_quant_gbs": next((kernels[n]["gbs"] for n in ("a4_smooth_quant_x", "quant_per_tensor_x",
+                                                           "rmsnorm_quant_x", "quant_bulk_x") if n in kernels), None),
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu_baseline, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
     }
@@ -431,6 +508,9 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=WORKLOAD,
                     help="the measured configuration is the 7B QKV prefill; the others are for profiling")
     ap.add_argument("--decode-m", type=int, default=16, choices=synth.DECODE_MS)
+    ap.add_argument("--variant", choices=sorted(VARIANTS), default="smoothquant",
+                    help="the measured path is smoothquant (per-token O1); the others measure the other "
+                         "activation granularities, the norm-folded form and the outlier decomposition")
     ap.add_argument("--e2e-steps", type=int, default=10, help="steps of the end-to-end measurement")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)

@@ -251,7 +251,7 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* x_scale, const int8_t* wq,
  *            starting from (float(acc_tn) * x_scale_t) * w_scale_n,
  *   every step an fp32 fused multiply-add, then rounded to out_dt.
  *   x_out [M x ld] and w_out [N x ld] float, device, 16-byte aligned, zero
- *   beyond the real outlier count; ld a multiple of 4 in [0, 64] (ld = 0 is
+ *   beyond the real outlier count; ld a multiple of 4 in [0, 32] (ld = 0 is
  *   the plain GEMM). out_dt SQ_F32 or SQ_BF16. Workspace and every other
  *   argument as for sq_w8a8_gemm. */
 sq_status sq_outlier_split(const float* xmax, int64_t K, float threshold, float* keep,

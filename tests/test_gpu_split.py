@@ -94,7 +94,7 @@ def _split_operands(M, N, K, ld, seed):
     return xq, wq, xs, wsc, xo, wo
 
 
-@pytest.mark.parametrize("M,N,K,ld", [(1, 300, 272, 4), (8, 4096, 1024, 8), (16, 1100, 4096, 64),
+@pytest.mark.parametrize("M,N,K,ld", [(1, 300, 272, 4), (8, 4096, 1024, 8), (16, 1100, 4096, 32),
                                       (100, 300, 272, 4), (128, 512, 1024, 16), (300, 1000, 1040, 8),
                                       (1024, 2048, 4096, 4)])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
@@ -117,6 +117,10 @@ def test_gemm_split_with_no_outliers_is_the_plain_gemm():
     with pytest.raises(sq.SqError) as err:
         sq.sq_w8a8_gemm_split(dev(xq), dev(xs), dev(wq), dev(wsc), dev(torch.zeros(200, 6)),
                               dev(torch.zeros(300, 6)), out_dtype=torch.float32)
+    assert err.value.status == sq.SQ_ERR_UNSUPPORTED
+    with pytest.raises(sq.SqError) as err:
+        sq.sq_w8a8_gemm_split(dev(xq), dev(xs), dev(wq), dev(wsc), dev(torch.zeros(200, 36)),
+                              dev(torch.zeros(300, 36)), out_dtype=torch.float32)
     assert err.value.status == sq.SQ_ERR_UNSUPPORTED
 
 

@@ -60,7 +60,8 @@ constexpr uint32_t IDESC_STREAM = make_idesc_i8(S_BM, S_BN);
 constexpr int STREAM_MAX_M = 16;
 
 enum OutKind { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
-constexpr int kMaxSplitLd = 64;  // outlier channels the decomposed epilogue takes
+constexpr int kMaxSplitLd = 32;  // outlier channels the decomposed epilogue takes
+constexpr size_t kSplitSmem = (size_t)BN * kMaxSplitLd * sizeof(float);   // w_out^T of one tile: 32 KB
 
 constexpr size_t tiled_smem_bytes() {
     return 1024 /*alignment slack*/ + STAGES * (A_STAGE + B_STAGE) + 256 /*barriers etc*/;
@@ -94,21 +95,49 @@ struct SplitTerm {
     int ld = 0;
 };
 
-// v[i] += sum_o x_out[row, o] * w_out[col0 + i, o] for the 32 columns of a row.
-// All lanes of a warp read the same w_out element at once (a broadcast).
-__device__ __forceinline__ void add_split32(float (&v)[32], int64_t row, int col0, int N, const SplitTerm& sp) {
-    const float* xr = sp.x_out + row * (int64_t)sp.ld;
+// The prefill kernels stage w_out of the tile's BN columns in shared memory,
+// transposed to [ld][BN], before each tile's epilogue (the four epilogue
+// warps together); every lane then reads the same float4 of four columns at
+// once (a broadcast). Two mbarriers with bounded waits order the staging:
+// SFULL (all four warps have written the tile) and SEMPTY (all four have
+// finished reading the previous one), so a warp that leaves early on an error
+// cannot strand the others.
+
+// Called by the four epilogue warps (threads 64..191) for their it-th tile.
+// Returns false if a wait gave up (the caller leaves its tile loop).
+__device__ __forceinline__ bool stage_split(float* w_s, const SplitTerm& sp, int nb, int N, uint32_t it,
+                                            uint32_t sfull, uint32_t sempty, long long limit,
+                                            volatile int* abort_flag) {
+    if (it > 0 && !mbar_wait(sempty, (it - 1) & 1, limit, abort_flag, SITE_GEMM_EPILOGUE)) return false;
+    const int n0 = nb * BN;
+    for (int i = (int)threadIdx.x - 64; i < BN * sp.ld; i += 128) {
+        const int o = i / BN, c = i - o * BN;
+        const int col = n0 + c;
+        w_s[o * BN + c] = col < N ? __ldg(sp.w_out + (int64_t)col * sp.ld + o) : 0.0f;
+    }
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(sfull);
+    return mbar_wait(sfull, it & 1, limit, abort_flag, SITE_GEMM_EPILOGUE);
+}
+
+// v[i] += sum_o x_out[row, o] * w_out[col0 + i, o] for 32 columns of a row;
+// xr = x_out + row * ld, ws_col = the staged w_out^T at column col0.
+__device__ __forceinline__ void add_split32(float (&v)[32], const float* __restrict__ xr, const float* ws_col,
+                                            int ld) {
 #pragma unroll 1
-    for (int o = 0; o < sp.ld; o += 4) {
-        const float4 xo = __ldg(reinterpret_cast<const float4*>(xr + o));
+    for (int o4 = 0; o4 < ld; o4 += 4) {
+        const float4 xo = __ldg(reinterpret_cast<const float4*>(xr + o4));
+        const float xv[4] = {xo.x, xo.y, xo.z, xo.w};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if (col0 + i < N) {
-                const float4 wo = __ldg(reinterpret_cast<const float4*>(sp.w_out + (int64_t)(col0 + i) * sp.ld + o));
-                v[i] = fmaf(xo.x, wo.x, v[i]);
-                v[i] = fmaf(xo.y, wo.y, v[i]);
-                v[i] = fmaf(xo.z, wo.z, v[i]);
-                v[i] = fmaf(xo.w, wo.w, v[i]);
+        for (int k = 0; k < 4; ++k) {
+            const float* wrow = ws_col + (o4 + k) * BN;
+#pragma unroll
+            for (int i4 = 0; i4 < 8; ++i4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(wrow + 4 * i4);
+                v[4 * i4] = fmaf(xv[k], w4.x, v[4 * i4]);
+                v[4 * i4 + 1] = fmaf(xv[k], w4.y, v[4 * i4 + 1]);
+                v[4 * i4 + 2] = fmaf(xv[k], w4.z, v[4 * i4 + 2]);
+                v[4 * i4 + 3] = fmaf(xv[k], w4.w, v[4 * i4 + 3]);
             }
         }
     }
@@ -133,7 +162,8 @@ __device__ __forceinline__ float add_split1(float v, int64_t t, int64_t n, const
 // Stores 32 consecutive outputs of one row (row-major y, row stride N).
 template <int OUT, bool SPLIT>
 __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int N, const uint32_t (&r)[32],
-                                            float sa, const float* __restrict__ w_scale, const SplitTerm& sp) {
+                                            float sa, const float* __restrict__ w_scale, const float* xr,
+                                            const float* ws_col, int ld) {
     const int64_t base = row * (int64_t)N + col0;
     const bool full = (col0 + 32 <= N);
     if (OUT == kOutI32) {
@@ -163,7 +193,7 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
         for (int i = 0; i < 32; ++i)
             v[i] = (col0 + i < N) ? dequant((int32_t)r[i], sa, __ldg(w_scale + col0 + i)) : 0.0f;
     }
-    if (SPLIT) add_split32(v, row, col0, N, sp);
+    if (SPLIT) add_split32(v, xr, ws_col, ld);
     if (OUT == kOutF32) {
         float* yp = static_cast<float*>(y) + base;
         if (full && (N & 3) == 0) {
@@ -216,6 +246,8 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const int FULL = 0, EMPTY = STAGES, TFULL = 2 * STAGES, TEMPTY = 2 * STAGES + 2, DRAIN = 2 * STAGES + 4;
+    // entry 2 * STAGES + 5 holds the TMEM address and the abort flag
+    const int SFULL = 2 * STAGES + 6, SEMPTY = 2 * STAGES + 7;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -227,6 +259,10 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             mbar_init(bar(TEMPTY + a), 4);
         }
         mbar_init(bar(DRAIN), 1);
+        if (SPLIT) {
+            mbar_init(bar(SFULL), 4);
+            mbar_init(bar(SEMPTY), 4);
+        }
         *abort_flag = 0;
         no_abort = 0;
         fence_barrier_init();
@@ -317,9 +353,12 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const int quarter = warp & 3;  // TMEM lanes this warp may read: 32*quarter ..
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        float* w_s = reinterpret_cast<float*>(smem + STAGES * (A_STAGE + B_STAGE) + 256);
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             int mb, nb;
             tile_coords(tile, num_m, num_n, mb, nb);
+            if (SPLIT && !stage_split(w_s, sp, nb, N, it, bar(SFULL), bar(SEMPTY), wait_limit, abort_flag)) break;
             if (!mbar_wait(bar(TFULL + acc), acc_phase, wait_limit, abort_flag, SITE_GEMM_EPILOGUE)) break;
             tc_fence_after();
             const int64_t row = (int64_t)mb * BM + quarter * 32 + lane;
@@ -333,12 +372,18 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
                 tmem_wait_ld();
                 const int col0 = nb * BN + c * 32;
-                if (row_ok && col0 < N) store_row32<OUT, SPLIT>(y, row, col0, N, r0, sa, w_scale, sp);
-                if (row_ok && col0 + 32 < N) store_row32<OUT, SPLIT>(y, row, col0 + 32, N, r1, sa, w_scale, sp);
+                const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
+                if (row_ok && col0 < N)
+                    store_row32<OUT, SPLIT>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
+                if (row_ok && col0 + 32 < N)
+                    store_row32<OUT, SPLIT>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(TEMPTY + acc));
+            if (lane == 0) {
+                mbar_arrive(bar(TEMPTY + acc));
+                if (SPLIT) mbar_arrive(bar(SEMPTY));   // this warp has read the staged tile
+            }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
@@ -450,6 +495,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const int FULL = 0, EMPTY = P_STAGES, TFULL = 2 * P_STAGES, TEMPTY = 2 * P_STAGES + 2, DRAIN = 2 * P_STAGES + 4;
+    // entry 2 * P_STAGES + 5 holds the TMEM address and the abort flag
+    const int SFULL = 2 * P_STAGES + 6, SEMPTY = 2 * P_STAGES + 7;   // this CTA's own staging
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < P_STAGES; ++s) {
@@ -461,6 +508,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             mbar_init(bar(TEMPTY + a), 8);   // 4 epilogue warps in each CTA
         }
         mbar_init(bar(DRAIN), 1);
+        if (SPLIT) {
+            mbar_init(bar(SFULL), 4);
+            mbar_init(bar(SEMPTY), 4);
+        }
         *abort_flag = 0;
         no_abort = 0;
         fence_barrier_init();
@@ -560,9 +611,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int quarter = warp & 3;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = pair; tile < num_tiles; tile += npairs) {
+        float* w_s = reinterpret_cast<float*>(smem + P_STAGES * (P_A_STAGE + P_B_STAGE) + 256);
+        uint32_t it = 0;
+        for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
             int mb, nb;
             tile_coords(tile, num_m, num_n, mb, nb);
+            if (SPLIT && !stage_split(w_s, sp, nb, N, it, bar(SFULL), bar(SEMPTY), wait_limit, abort_flag)) break;
             if (!mbar_wait(bar(TFULL + acc), acc_phase, wait_limit, abort_flag, SITE_GEMM_EPILOGUE)) break;
             tc_fence_after();
             const int64_t row = (int64_t)mb * 256 + rank * 128 + quarter * 32 + lane;
@@ -576,14 +630,18 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
                 tmem_wait_ld();
                 const int col0 = nb * BN + c * 32;
-                if (row_ok && col0 < N) store_row32<OUT, SPLIT>(y, row, col0, N, r0, sa, w_scale, sp);
-                if (row_ok && col0 + 32 < N) store_row32<OUT, SPLIT>(y, row, col0 + 32, N, r1, sa, w_scale, sp);
+                const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
+                if (row_ok && col0 < N)
+                    store_row32<OUT, SPLIT>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
+                if (row_ok && col0 + 32 < N)
+                    store_row32<OUT, SPLIT>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 if (rank == 0) mbar_arrive(bar(TEMPTY + acc));
                 else arrive_on_cta0(bar(TEMPTY + acc));
+                if (SPLIT) mbar_arrive(bar(SEMPTY));   // this warp has read the staged tile
             }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
@@ -864,7 +922,7 @@ sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float
                        int M, int N, int K, cudaStream_t st, const SplitTerm& sp = SplitTerm{}) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
-    const size_t smem = tiled_smem_bytes();
+    const size_t smem = tiled_smem_bytes() + (SPLIT ? kSplitSmem : 0);
     sq_status r = ensure_smem_attr(gemm_tiled_kernel<OUT, SPLIT>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
@@ -878,7 +936,7 @@ sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float*
                       int M, int N, int K, cudaStream_t st, const SplitTerm& sp = SplitTerm{}) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
-    const size_t smem = pair_smem_bytes();
+    const size_t smem = pair_smem_bytes() + (SPLIT ? kSplitSmem : 0);
     sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT, SPLIT>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const int tiles = ((M + 255) / 256) * ((N + 255) / 256);

@@ -275,12 +275,16 @@ def sq_w8a8_gemm_noalloc(xq: torch.Tensor, x_scale: torch.Tensor | None, wq: tor
     return y
 
 
-def sq_outlier_split(xmax: torch.Tensor, threshold: float, stream=None):
+def sq_outlier_split(xmax: torch.Tensor, threshold: float, keep: torch.Tensor | None = None,
+                     idx: torch.Tensor | None = None, count: torch.Tensor | None = None, stream=None):
     """-> (keep float32 [K], idx int32 [K] (first `count` valid), count int32 [1]), all on the device."""
     K = xmax.shape[0]
-    keep = torch.empty(K, dtype=torch.float32, device=xmax.device)
-    idx = torch.empty(max(K, 1), dtype=torch.int32, device=xmax.device)
-    count = torch.empty(1, dtype=torch.int32, device=xmax.device)
+    if keep is None:
+        keep = torch.empty(K, dtype=torch.float32, device=xmax.device)
+    if idx is None:
+        idx = torch.empty(max(K, 1), dtype=torch.int32, device=xmax.device)
+    if count is None:
+        count = torch.empty(1, dtype=torch.int32, device=xmax.device)
     _check(_lib.sq_outlier_split(_dev(xmax, "xmax"), K, float(threshold), _dev(keep, "keep"), _dev(idx, "idx"),
                                  _dev(count, "count"), _stream(stream)), "sq_outlier_split")
     return keep, idx, count
