@@ -218,6 +218,8 @@ VARIANTS = {
     "per_tensor_static": "a1(X) a1(W) a2 a3, static range from the calibration maxima, per-tensor codes, a5 (O3)",
     "rmsnorm": "a1(X) a1(W) a2 a3, gain fold, RMSNorm + per-token codes, a5 (the norm-folded O1)",
     "split": "a1(X), outlier split, bulk int8 of W and X, outlier gathers, int8 GEMM + fp32 outlier epilogue",
+    "alpha_search": "one sq_alpha_search call: a1(X) a1(W), the float reference product, then per alpha "
+                    "a2 a3 a4 a5 (fp32 out) and the error reduction",
 }
 SPLIT_THRESHOLD = 6.0  # outlier channels: calibration maximum >= 6 (the synthetic outliers are 20-80x)
 
@@ -241,6 +243,20 @@ def build_step(variant, sq, wl, x, w, dev, stream):
     ops = 2.0 * M * N * K
     gemm_bytes = M * K + N * K + M * 4 + N * 4 + M * N * out_es
     st = []
+    if variant == "alpha_search":
+        alphas = list(synth.DOWN_70B_ALPHAS)
+        sws = torch.zeros(sq.sq_alpha_search_workspace_size(M, N, K, len(alphas)), dtype=torch.uint8, device=dev)
+        once = M * K * in_es + N * K * in_es + 8 * K + (M * K + N * K) * in_es + 4 * M * N
+        per_alpha = (12 * K + N * K * in_es + N * K + 4 * N + M * K * in_es + M * K + 4 * M
+                     + M * K + N * K + 4 * (M + N) + 4 * M * N + 8 * M * N)
+        result = {}
+
+        def search():
+            errs, best = sq.sq_alpha_search(x, w, alphas, workspace=sws, stream=stream)
+            result.update(errors=[round(e, 6) for e in errs], best_alpha=best)
+        st.append(("alpha_search", search, once + len(alphas) * per_alpha, len(alphas) * ops))
+        return maxima, st, {"alphas": alphas, "search": result,
+                            "note": "the call synchronizes its stream; ops = int8 GEMM ops over all alphas"}
     st.append(("a1_calibrate_x", lambda: sq.sq_calibrate_absmax(x, xmax, stream=stream), M * K * in_es + K * 4, 0))
     if variant == "split":
         keep = torch.empty(K, dtype=torch.float32, device=dev)
@@ -385,10 +401,24 @@ def run_ours(args, world, rank, local):
             tops = ops / (ms * 1e-3) / 1e12
             entry.update({"tops": round(tops, 1), "tensor_frac": round(tops / int8_peak, 3)})
         kernels[n] = entry
-    gemm_ms = per_kernel["a5_w8a8_gemm"]
-    achieved = ops / (gemm_ms * 1e-3) / 1e12
+    if args.variant == "alpha_search":
+        ms = per_kernel["alpha_search"]
+        n_a = len(variant_info["alphas"])
+        value = world * n_a * ops / (step_ms_max * 1e-3) / 1e12
+        gbs = kb["alpha_search"] / (ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "the whole search (memory-bound passes dominate; the int8 and "
+                                              "reference GEMMs are included in the time)",
+                    "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                    "traffic": None, "peak_source": f"{peak_src}: hbm_gbs",
+                    "algorithmic_bytes_per_launch": kb["alpha_search"]}
+        kernels["alpha_search"]["per_alpha_ms"] = round(ms / n_a, 4)
+    else:
+        gemm_ms = per_kernel["a5_w8a8_gemm"]
+        achieved = ops / (gemm_ms * 1e-3) / 1e12
     default_gemm = args.variant != "split"
-    if M > 16:
+    if args.variant == "alpha_search":
+        pass
+    elif M > 16:
         roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel (a5, paired-SM tcgen05)" if M > 128
                     else "gemm_tiled_kernel (a5)",
                     "achieved": round(achieved, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
