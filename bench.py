@@ -213,7 +213,8 @@ def workload_inputs(name: str, decode_m: int):
 
 
 VARIANTS = {
-    "smoothquant": "a1(X) a1(W) a2 a3 a4 a5: per-token dynamic activation scales (O1)",
+    "smoothquant": "a1(X)+a1(W) in one launch, a2, a3, a4, a5: per-token dynamic activation scales (O1)",
+    "smoothquant_steps": "a1(X) a1(W) a2 a3 a4 a5, one launch per step (per-step timings)",
     "per_tensor_dynamic": "a1(X) a1(W) a2 a3, per-tensor range of X/s, per-tensor codes, a5 (O2)",
     "per_tensor_static": "a1(X) a1(W) a2 a3, static range from the calibration maxima, per-tensor codes, a5 (O3)",
     "rmsnorm": "a1(X) a1(W) a2 a3, gain fold, RMSNorm + per-token codes, a5 (the norm-folded O1)",
@@ -257,6 +258,18 @@ def build_step(variant, sq, wl, x, w, dev, stream):
         st.append(("alpha_search", search, once + len(alphas) * per_alpha, len(alphas) * ops))
         return maxima, st, {"alphas": alphas, "search": result,
                             "note": "the call synchronizes its stream; ops = int8 GEMM ops over all alphas"}
+    if variant == "smoothquant":
+        st.append(("a1_calibrate_xw", lambda: sq.sq_calibrate_absmax_pair(x, w, xmax, wmax, stream=stream),
+                   (M + N) * K * in_es + 2 * K * 4, 0))
+        st.append(("a2_smooth_factors", lambda: sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream),
+                   3 * K * 4, 0))
+        st.append(("a3_fold_quant_w", lambda: sq.sq_fold_quant_weights(w, s, wq=wq, w_scale=wsc, stream=stream),
+                   N * K * in_es + K * 4 + N * K + N * 4, 0))
+        st.append(("a4_smooth_quant_x", lambda: sq.sq_smooth_quant_act(x, s, xq=xq, x_scale=xsc, stream=stream),
+                   M * K * in_es + K * 4 + M * K + M * 4, 0))
+        st.append(("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm(xq, xsc, wq, wsc, y=y, workspace=gws, stream=stream),
+                   gemm_bytes, ops))
+        return maxima, st, {}
     st.append(("a1_calibrate_x", lambda: sq.sq_calibrate_absmax(x, xmax, stream=stream), M * K * in_es + K * 4, 0))
     if variant == "split":
         keep = torch.empty(K, dtype=torch.float32, device=dev)
@@ -291,7 +304,7 @@ def build_step(variant, sq, wl, x, w, dev, stream):
                N * K * in_es + K * 4 + N * K + N * 4, 0))
     act_bytes = M * K * in_es + K * 4 + M * K + M * 4
     extra = {}
-    if variant == "smoothquant":
+    if variant == "smoothquant_steps":
         st.append(("a4_smooth_quant_x", lambda: sq.sq_smooth_quant_act(x, s, xq=xq, x_scale=xsc, stream=stream),
                    act_bytes, 0))
     elif variant == "per_tensor_dynamic":
@@ -484,6 +497,8 @@ def run_ours(args, world, rank, local):
                    "variant": args.variant, "step": VARIANTS[args.variant] + ", one stream", **variant_info},
         "act_quant_gbs": next((kernels[n]["gbs"] for n in ("a4_smooth_quant_x", "quant_per_tensor_x",
                                                            "rmsnorm_quant_x", "quant_bulk_x") if n in kernels), None),
+        "act_quant_gbs_from": next((n for n in ("a4_smooth_quant_x", "quant_per_tensor_x",
+                                                "rmsnorm_quant_x", "quant_bulk_x") if n in kernels), None),
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu_baseline, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
     }

@@ -129,6 +129,15 @@ sq_status sq_smooth_quant_act(const void* x, sq_dtype dt, int64_t T, int64_t K,
                               const float* s, int8_t* xq, float* x_scale,
                               sq_stream_t stream);
 
+/* ---------------------------------------------------------------- both calibrations in one launch
+ * sq_calibrate_absmax_pair: step a1 on the activations x [T x K] into xmax and
+ * on the weights w [N x K] into wmax (both running maxima, as
+ * sq_calibrate_absmax), in one launch whose blocks are shared between the two
+ * tensors, so neither waits for the tail of the other. Same results as the two
+ * separate calls, bit for bit. Same dtype for both. */
+sq_status sq_calibrate_absmax_pair(const void* x, int64_t T, const void* w, int64_t N, sq_dtype dt,
+                                   int64_t K, float* xmax, float* wmax, sq_stream_t stream);
+
 /* ---------------------------------------------------------------- per-tensor scales (O2, O3)
  * One activation scale for the whole tensor instead of one per token: the
  * per-tensor dynamic (O2) and per-tensor static (O3) levels of "SmoothQuant

@@ -247,6 +247,57 @@ def test_gemm_decode_workspace_reuse():
     assert int(ws.count_nonzero()) == 0
 
 
+# ------------------------------------------------------------------ fused launches
+PAIR_SHAPES = [(1, 3, 16), (5, 300, 48), (130, 40, 1040), (64, 12288 // 8, 4096), (17, 333, 5120), (4, 9, 28672),
+               (3, 2, 65536), (0, 7, 1040), (7, 0, 1040)]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("T,N,K", PAIR_SHAPES)
+def test_fused_calibration_equals_separate_calls(dtype, T, N, K):
+    """sq_calibrate_absmax_pair gives the separate calls' results (and the
+    oracle's) bit for bit; the quantization steps follow on its maxima."""
+    x = outlier_x(max(T, 1), K, dtype, seed=T * 11 + K)[:T]
+    w = rand_w(max(N, 1), K, dtype, seed=N * 13 + K)[:N]
+    if T > 2:
+        x[1] = 0
+    xd, wd = dev(x), dev(w)
+    xmax = torch.zeros(K, dtype=torch.float32, device=DEV)
+    wmax = torch.zeros(K, dtype=torch.float32, device=DEV)
+    sq.sq_calibrate_absmax_pair(xd, wd, xmax, wmax)
+    hx, hw = synth.host_array(x), synth.host_array(w)
+    o_xmax = oracle.col_absmax(hx) if T else np.zeros(K, np.float32)
+    o_wmax = oracle.col_absmax(hw) if N else np.zeros(K, np.float32)
+    assert_bitexact_f32(host(xmax), o_xmax, "paired xmax")
+    assert_bitexact_f32(host(wmax), o_wmax, "paired wmax")
+    s = _s_for(K, K + 5)
+    sd = dev(torch.from_numpy(s))
+    wq, wsc = sq.sq_fold_quant_weights(wd, sd)
+    xq, xs = sq.sq_smooth_quant_act(xd, sd)
+    if N:
+        oq, osc = oracle.fold_quant_weights(hw, s)
+        assert_equal(host(wq), oq, "paired wq")
+        assert_bitexact_f32(host(wsc), osc, "paired w_scale")
+    if T:
+        oq, osc = oracle.smooth_quant_act(hx, s)
+        assert_equal(host(xq), oq, "paired xq")
+        assert_bitexact_f32(host(xs), osc, "paired x_scale")
+    assert sq.sq_get_status() == sq.SQ_OK
+
+
+def test_fused_calibration_full_size_qkv():
+    wl = synth.WORKLOADS["qkv_prefill_7b"]
+    x, w = synth.make(wl.name)
+    xd, wd = dev(x), dev(w)
+    K = wl.K
+    m1 = torch.zeros(2 * K, dtype=torch.float32, device=DEV)
+    m2 = torch.zeros(2 * K, dtype=torch.float32, device=DEV)
+    sq.sq_calibrate_absmax_pair(xd, wd, m1[:K], m1[K:])
+    sq.sq_calibrate_absmax(xd, m2[:K])
+    sq.sq_calibrate_absmax(wd, m2[K:])
+    assert torch.equal(m1, m2)
+
+
 # ------------------------------------------------------------------ whole path
 def _check_path(x, w, alpha, out_dtype, rows=None, calib=None):
     """Run every step on the GPU and compare each output with the oracle;

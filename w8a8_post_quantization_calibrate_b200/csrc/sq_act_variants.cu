@@ -162,10 +162,10 @@ sq_status tensor_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_t c
     if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
     if (dt == SQ_F32)
         col_absmax_kernel<float, true><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, amax, s);
+            static_cast<const uint8_t*>(x), rows, cols, per, amax, s, AbsmaxPair{});
     else
         col_absmax_kernel<__nv_bfloat16, true><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, amax, s);
+            static_cast<const uint8_t*>(x), rows, cols, per, amax, s, AbsmaxPair{});
     return check_launch("col_absmax_kernel<tensor>");
 }
 

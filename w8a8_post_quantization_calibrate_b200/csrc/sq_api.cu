@@ -121,6 +121,8 @@ sq_status fold_quant_weights_impl(const void*, sq_dtype, int64_t, int64_t, const
                                   cudaStream_t);
 sq_status smooth_quant_act_impl(const void*, sq_dtype, int64_t, int64_t, const float*, int8_t*, float*,
                                 cudaStream_t);
+sq_status calibrate_absmax_pair_impl(const void*, int64_t, const void*, int64_t, sq_dtype, int64_t, float*, float*,
+                                     cudaStream_t);
 
 sq_status linear_impl(const void* x, const void* w, sq_dtype in_dt, int64_t M, int64_t N, int64_t K,
                       float alpha, float eps, void* y, sq_dtype out_dt, void* ws, size_t ws_bytes,
@@ -169,8 +171,7 @@ sq_status linear_impl(const void* x, const void* w, sq_dtype in_dt, int64_t M, i
     // xmax and wmax are adjacent: one memset starts both calibrations from +0.
     if ((e = cudaMemsetAsync(xmax, 0, L.s - L.xmax, st)) != cudaSuccess) return cuda_fail(e, "clear maxima");
     sq_status r;
-    if ((r = calibrate_absmax_impl(xd, in_dt, M, K, xmax, st)) != SQ_OK) return r;
-    if ((r = calibrate_absmax_impl(wd, in_dt, N, K, wmax, st)) != SQ_OK) return r;
+    if ((r = calibrate_absmax_pair_impl(xd, M, wd, N, in_dt, K, xmax, wmax, st)) != SQ_OK) return r;
     if ((r = smooth_factors_impl(xmax, wmax, K, alpha, eps, s, st)) != SQ_OK) return r;
     if ((r = fold_quant_weights_impl(wd, in_dt, N, K, s, wq, wsc, st)) != SQ_OK) return r;
     if ((r = smooth_quant_act_impl(xd, in_dt, M, K, s, xq, xs, st)) != SQ_OK) return r;

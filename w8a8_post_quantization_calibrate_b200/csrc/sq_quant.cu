@@ -51,6 +51,15 @@ struct Vec16<__nv_bfloat16> {
 constexpr int kAbsmaxThreads = 256;
 constexpr int kAbsmaxRowsInFlight = 8;   // per warp; a block covers 64 rows per iteration
 
+// Two tensors in one launch (the activations and the weights of a layer share
+// K): row-chunk blocks [0, rc1) read the first, the others the second.
+struct AbsmaxPair {
+    const uint8_t* x2 = nullptr;
+    int64_t rows2 = 0, per2 = 0;
+    float* absmax2 = nullptr;
+    int rc1 = 0;   // 0: one tensor
+};
+
 // TENSOR = true: the per-tensor variant. Each column maximum is first divided
 // by s_j (RN(max|x| / s_j) = max |RN(x / s_j)| for s_j > 0, because rounding
 // is monotone), the block's columns are reduced to one value, and that value
@@ -58,12 +67,21 @@ constexpr int kAbsmaxRowsInFlight = 8;   // per warp; a block covers 64 rows per
 template <typename T, bool TENSOR>
 __global__ void __launch_bounds__(kAbsmaxThreads)
 col_absmax_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t cols,
-                  int64_t rows_per_chunk, float* __restrict__ absmax, const float* __restrict__ s) {
+                  int64_t rows_per_chunk, float* __restrict__ absmax, const float* __restrict__ s,
+                  const AbsmaxPair pair) {
     constexpr int VEC = Vec16<T>::N;
     constexpr int TILE = 32 * VEC;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int64_t chunk = blockIdx.y;
+    if (pair.rc1 > 0 && (int)blockIdx.y >= pair.rc1) {
+        x = pair.x2;
+        rows = pair.rows2;
+        rows_per_chunk = pair.per2;
+        absmax = pair.absmax2;
+        chunk -= pair.rc1;
+    }
     const int64_t col = (int64_t)blockIdx.x * TILE + lane * VEC;
-    const int64_t r_begin = (int64_t)blockIdx.y * rows_per_chunk;
+    const int64_t r_begin = chunk * rows_per_chunk;
     const int64_t r_end = min(rows, r_begin + rows_per_chunk);
     const int64_t row_bytes = cols * (int64_t)sizeof(T);
 
@@ -795,11 +813,61 @@ sq_status calibrate_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_
     if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
     if (dt == SQ_F32)
         col_absmax_kernel<float, false><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, absmax, nullptr);
+            static_cast<const uint8_t*>(x), rows, cols, per, absmax, nullptr, AbsmaxPair{});
     else
         col_absmax_kernel<__nv_bfloat16, false><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, absmax, nullptr);
+            static_cast<const uint8_t*>(x), rows, cols, per, absmax, nullptr, AbsmaxPair{});
     return check_launch("col_absmax_kernel");
+}
+
+// Both calibrations of a layer in one launch: one wave of blocks shared between
+// the activations and the weights in proportion to their rows.
+sq_status calibrate_absmax_pair_impl(const void* x, int64_t T, const void* w, int64_t N, sq_dtype dt, int64_t K,
+                                     float* xmax, float* wmax, cudaStream_t st) {
+    sq_status r;
+    if ((r = check_input_dtype(dt)) != SQ_OK) return r;
+    if ((r = check_matrix(x, T, K, "x")) != SQ_OK) return r;
+    if ((r = check_matrix(w, N, K, "w")) != SQ_OK) return r;
+    if (K > 0 && (!xmax || !wmax)) { set_error("absmax: NULL pointer"); return SQ_ERR_INVALID_ARG; }
+    if (K == 0) return SQ_OK;
+    if (T == 0) return calibrate_absmax_impl(w, dt, N, K, wmax, st);
+    if (N == 0) return calibrate_absmax_impl(x, dt, T, K, xmax, st);
+    const int es = dt == SQ_F32 ? 4 : 2;
+    const int64_t tile = 32 * (16 / es);
+    const int64_t ct = (K + tile - 1) / tile;
+    if (ct > 2147483647LL) { set_error("cols too large"); return SQ_ERR_UNSUPPORTED; }
+    const int64_t step_rows = 8 * kAbsmaxRowsInFlight;
+    const int64_t target = (int64_t)device_info().sm_count * 8;
+    auto chunks = [&](int64_t rows, int64_t share, int64_t& per) {
+        int64_t rc = share / ct;
+        if (rc < 1) rc = 1;
+        per = (rows + rc - 1) / rc;
+        per = (per + step_rows - 1) / step_rows * step_rows;
+        return (rows + per - 1) / per;
+    };
+    int64_t per_x = 0, per_w = 0;
+    const int64_t share_x = target * T / (T + N);
+    const int64_t rc_x = chunks(T, share_x, per_x);
+    const int64_t rc_w = chunks(N, target - share_x, per_w);
+    if (rc_x + rc_w > 65535) {
+        // very tall inputs: one launch per tensor
+        if ((r = calibrate_absmax_impl(x, dt, T, K, xmax, st)) != SQ_OK) return r;
+        return calibrate_absmax_impl(w, dt, N, K, wmax, st);
+    }
+    AbsmaxPair pair;
+    pair.x2 = static_cast<const uint8_t*>(w);
+    pair.rows2 = N;
+    pair.per2 = per_w;
+    pair.absmax2 = wmax;
+    pair.rc1 = (int)rc_x;
+    const dim3 grid((unsigned)ct, (unsigned)(rc_x + rc_w));
+    if (dt == SQ_F32)
+        col_absmax_kernel<float, false><<<grid, kAbsmaxThreads, 0, st>>>(
+            static_cast<const uint8_t*>(x), T, K, per_x, xmax, nullptr, pair);
+    else
+        col_absmax_kernel<__nv_bfloat16, false><<<grid, kAbsmaxThreads, 0, st>>>(
+            static_cast<const uint8_t*>(x), T, K, per_x, xmax, nullptr, pair);
+    return check_launch("col_absmax_kernel<pair>");
 }
 
 sq_status smooth_factors_impl(const float* xmax, const float* wmax, int64_t K, float alpha,
@@ -844,6 +912,12 @@ sq_status smooth_quant_act_impl(const void* x, sq_dtype dt, int64_t T, int64_t K
 }  // namespace sq
 
 extern "C" {
+
+sq_status sq_calibrate_absmax_pair(const void* x, int64_t T, const void* w, int64_t N, sq_dtype dt, int64_t K,
+                                   float* xmax, float* wmax, sq_stream_t stream) {
+    return sq::calibrate_absmax_pair_impl(x, T, w, N, dt, K, xmax, wmax, (cudaStream_t)stream);
+}
+
 
 sq_status sq_calibrate_absmax(const void* x, sq_dtype dt, int64_t rows, int64_t cols,
                               float* absmax, sq_stream_t stream) {

@@ -216,8 +216,7 @@ sq_status alpha_search_impl(const void* x, const void* w, sq_dtype dt, int64_t T
     if ((e = cudaMemcpyAsync(alphas_d, alphas, (size_t)n_alpha * sizeof(float), cudaMemcpyHostToDevice, st)) != cudaSuccess)
         return cuda_fail(e, "copy alphas");
     if ((e = cudaMemsetAsync(xmax, 0, L.s - L.xmax, st)) != cudaSuccess) return cuda_fail(e, "clear maxima");
-    if ((r = calibrate_absmax_impl(x, dt, T, K, xmax, st)) != SQ_OK) return r;
-    if ((r = calibrate_absmax_impl(w, dt, N, K, wmax, st)) != SQ_OK) return r;
+    if ((r = calibrate_absmax_pair_impl(x, T, w, N, dt, K, xmax, wmax, st)) != SQ_OK) return r;
     if ((r = reference_gemm(x, w, dt, T, N, K, yref, st)) != SQ_OK) return r;
     const int64_t nel = T * N;
     int blocks = device_info().sm_count * 4;

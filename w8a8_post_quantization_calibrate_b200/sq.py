@@ -43,6 +43,7 @@ _SIGS = {
     "sq_smooth_factors": ([_vp, _vp, _i64, _f32, _f32, _vp, _vp], _int),
     "sq_fold_quant_weights": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_smooth_quant_act": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "sq_calibrate_absmax_pair": ([_vp, _i64, _vp, _i64, _int, _i64, _vp, _vp, _vp], _int),
     "sq_tensor_absmax": ([_vp, _int, _i64, _i64, _vp, _vp, _vp], _int),
     "sq_quant_act_per_tensor": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp], _int),
     "sq_fold_norm_gain": ([_vp, _int, _i64, _vp, _vp, _vp], _int),
@@ -159,6 +160,18 @@ def sq_smooth_quant_act(x: torch.Tensor, s: torch.Tensor, xq: torch.Tensor | Non
     _check(_lib.sq_smooth_quant_act(_dev(x, "x"), _dt(x), T, K, _dev(s, "s"), _dev(xq, "xq"),
                                     _dev(x_scale, "x_scale"), _stream(stream)), "sq_smooth_quant_act")
     return xq, x_scale
+
+
+def sq_calibrate_absmax_pair(x: torch.Tensor, w: torch.Tensor, xmax: torch.Tensor, wmax: torch.Tensor,
+                             stream=None):
+    """Running column maxima of x into xmax and of w into wmax, one launch."""
+    T, K = x.shape
+    N = w.shape[0]
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must have the same dtype")
+    _check(_lib.sq_calibrate_absmax_pair(_dev(x, "x"), T, _dev(w, "w"), N, _dt(x), K, _dev(xmax, "xmax"),
+                                         _dev(wmax, "wmax"), _stream(stream)), "sq_calibrate_absmax_pair")
+    return xmax, wmax
 
 
 def _opt_dev(t: torch.Tensor | None, name: str):
