@@ -53,6 +53,8 @@ per_tensor_quant_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t col
     const int64_t r_begin = (int64_t)blockIdx.y * rows_per_chunk;
     const int64_t r_end = min(rows, r_begin + rows_per_chunk);
 
+    pdl_wait();
+    pdl_trigger();
     const float amax = *amax_p;
     const bool zero = !(amax > 0.0f);
     const float scale = zero ? 1.0f : __fdiv_rn(amax, 127.0f);
@@ -161,12 +163,10 @@ sq_status tensor_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_t c
     int64_t per = 0;
     if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
     if (dt == SQ_F32)
-        col_absmax_kernel<float, true><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, amax, s, AbsmaxPair{});
-    else
-        col_absmax_kernel<__nv_bfloat16, true><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, amax, s, AbsmaxPair{});
-    return check_launch("col_absmax_kernel<tensor>");
+        return launch_pdl("col_absmax_kernel<tensor>", col_absmax_kernel<float, true>, grid, dim3(kAbsmaxThreads), 0,
+                          st, 1, static_cast<const uint8_t*>(x), rows, cols, per, amax, s, AbsmaxPair{});
+    return launch_pdl("col_absmax_kernel<tensor>", col_absmax_kernel<__nv_bfloat16, true>, grid, dim3(kAbsmaxThreads),
+                      0, st, 1, static_cast<const uint8_t*>(x), rows, cols, per, amax, s, AbsmaxPair{});
 }
 
 sq_status quant_act_per_tensor_impl(const void* x, sq_dtype dt, int64_t T, int64_t K, const float* s,
@@ -182,12 +182,10 @@ sq_status quant_act_per_tensor_impl(const void* x, sq_dtype dt, int64_t T, int64
     int64_t per = 0;
     if ((r = absmax_grid(T, K, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
     if (dt == SQ_F32)
-        per_tensor_quant_kernel<float><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), T, K, per, s, amax, xq, x_scale);
-    else
-        per_tensor_quant_kernel<__nv_bfloat16><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), T, K, per, s, amax, xq, x_scale);
-    return check_launch("per_tensor_quant_kernel");
+        return launch_pdl("per_tensor_quant_kernel", per_tensor_quant_kernel<float>, grid, dim3(kAbsmaxThreads), 0, st,
+                          1, static_cast<const uint8_t*>(x), T, K, per, s, amax, xq, x_scale);
+    return launch_pdl("per_tensor_quant_kernel", per_tensor_quant_kernel<__nv_bfloat16>, grid, dim3(kAbsmaxThreads), 0,
+                      st, 1, static_cast<const uint8_t*>(x), T, K, per, s, amax, xq, x_scale);
 }
 
 sq_status fold_norm_gain_impl(const void* g, sq_dtype dt, int64_t K, const float* s, float* gf,

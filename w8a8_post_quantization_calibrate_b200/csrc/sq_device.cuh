@@ -87,6 +87,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
     }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// The library's kernels are launched with programmatic stream serialization:
+// a kernel may be scheduled while the previous kernel in the stream is still
+// finishing. Every kernel calls pdl_wait() before its first access to global
+// memory (it returns once the previous grid has completed and its writes are
+// visible; immediately if there is no such grid), then pdl_trigger() so that
+// the next kernel can be scheduled in turn. Only shared-memory and TMEM set-up
+// may come before pdl_wait().
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion signalled on `bar`
 // (complete_tx). No multicast. x is the innermost (contiguous) coordinate.

@@ -278,6 +278,8 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
@@ -529,6 +531,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer (both CTAs)
@@ -716,6 +720,8 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -927,8 +933,8 @@ sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float
     if (r != SQ_OK) return r;
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = tiles < di.sm_count ? tiles : di.sm_count;
-    gemm_tiled_kernel<OUT, SPLIT><<<grid, GEMM_THREADS, smem, st>>>(ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
-    return check_launch("gemm_tiled_kernel");
+    return launch_pdl("gemm_tiled_kernel", gemm_tiled_kernel<OUT, SPLIT>, dim3(grid), dim3(GEMM_THREADS), smem, st, 1,
+                      ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
 }
 
 template <int OUT, bool SPLIT = false>
@@ -942,22 +948,8 @@ sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float*
     const int tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int max_pairs = di.sm_count / 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<OUT, SPLIT>, ta, tb, xs, wsc, y, M, N, K, sp,
-                                       wait_limit_cycles());
-    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(gemm_pair_kernel)");
-    return check_launch("gemm_pair_kernel");
+    return launch_pdl("gemm_pair_kernel", gemm_pair_kernel<OUT, SPLIT>, dim3(2 * pairs), dim3(GEMM_THREADS), smem, st,
+                      2, ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
 }
 
 template <int OUT, bool SPLIT = false>
@@ -971,9 +963,8 @@ sq_status launch_stream(const CUtensorMap& tw, const CUtensorMap& tx, const floa
     if (r != SQ_OK) return r;
     const long long units = (long long)((N + S_BM - 1) / S_BM) * ((K + BK - 1) / BK);
     const int grid = units < di.sm_count ? (int)units : di.sm_count;
-    gemm_stream_kernel<OUT, SPLIT><<<grid, GEMM_THREADS, smem, st>>>(tw, tx, xs, wsc, y, M, N, K, ws_acc, counts,
-                                                                     sp, wait_limit_cycles());
-    return check_launch("gemm_stream_kernel");
+    return launch_pdl("gemm_stream_kernel", gemm_stream_kernel<OUT, SPLIT>, dim3(grid), dim3(GEMM_THREADS), smem, st,
+                      1, tw, tx, xs, wsc, y, M, N, K, ws_acc, counts, sp, wait_limit_cycles());
 }
 
 size_t stream_ws_bytes(int64_t M, int64_t N) {

@@ -71,6 +71,8 @@ col_absmax_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t cols,
                   const AbsmaxPair pair) {
     constexpr int VEC = Vec16<T>::N;
     constexpr int TILE = 32 * VEC;
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int64_t chunk = blockIdx.y;
     if (pair.rc1 > 0 && (int)blockIdx.y >= pair.rc1) {
@@ -148,6 +150,8 @@ __device__ __forceinline__ double pow_alpha_dev(double v, double a) {
 
 __global__ void smooth_factors_kernel(const float* __restrict__ xmax, const float* __restrict__ wmax,
                                       int64_t K, float alpha, float eps, float* __restrict__ s) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= K) return;
     const float xm = xmax[j] > eps ? xmax[j] : eps;
@@ -203,6 +207,8 @@ row_quant_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float*
                  int8_t* __restrict__ q, float* __restrict__ scale_out) {
     constexpr int NW = TPB / 32;
     __shared__ float red[2][NW];
+    pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t nchunks = K >> 3;
     int parity = 0;
@@ -458,6 +464,8 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
     const int grp = warp / R, wig = warp % R;
     const int gl = wig * 32 + lane;          // lane index inside the group
 
+    pdl_wait();
+    pdl_trigger();
     for (int64_t c = threadIdx.x; c < nchunks; c += blockDim.x) {
         float4 a = __ldg(reinterpret_cast<const float4*>(s + c * 8));
         float4 b = __ldg(reinterpret_cast<const float4*>(s + c * 8 + 4));
@@ -653,9 +661,8 @@ sq_status launch_row_quant_inst(const void* in, int64_t rows, int64_t K, const f
                                 int8_t* q, float* scale, cudaStream_t st) {
     const int64_t max_blocks = (int64_t)device_info().sm_count * (2048 / TPB);
     const int grid = (int)(rows < max_blocks ? rows : max_blocks);
-    row_quant_kernel<T, MODE, TPB, MAXC><<<grid, TPB, 0, st>>>(
-        static_cast<const T*>(in), rows, K, s, q, scale);
-    return check_launch("row_quant_kernel");
+    return launch_pdl("row_quant_kernel", row_quant_kernel<T, MODE, TPB, MAXC>, dim3(grid), dim3(TPB), 0, st, 1,
+                      static_cast<const T*>(in), rows, K, s, q, scale);
 }
 
 template <typename T, int MODE, int TPB>
@@ -700,8 +707,8 @@ sq_status launch_row_quant_fast_inst(const void* in, int64_t rows, int64_t K, co
     const int64_t need = (rows + groups - 1) / groups;
     const int64_t max_blocks = (int64_t)di.sm_count * per_sm;
     const int grid = (int)(need < max_blocks ? need : max_blocks);
-    kern<<<grid, threads, smem, st>>>(static_cast<const T*>(in), rows, K, s, q, scale, eps, r_out);
-    return check_launch("row_quant_fast_kernel");
+    return launch_pdl("row_quant_fast_kernel", kern, dim3(grid), dim3(threads), smem, st, 1,
+                      static_cast<const T*>(in), rows, K, s, q, scale, eps, r_out);
 }
 
 template <typename T, int MODE>
@@ -812,12 +819,11 @@ sq_status calibrate_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_
     int64_t per = 0;
     if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
     if (dt == SQ_F32)
-        col_absmax_kernel<float, false><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, absmax, nullptr, AbsmaxPair{});
-    else
-        col_absmax_kernel<__nv_bfloat16, false><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), rows, cols, per, absmax, nullptr, AbsmaxPair{});
-    return check_launch("col_absmax_kernel");
+        return launch_pdl("col_absmax_kernel", col_absmax_kernel<float, false>, grid, dim3(kAbsmaxThreads), 0, st, 1,
+                          static_cast<const uint8_t*>(x), rows, cols, per, absmax, (const float*)nullptr,
+                          AbsmaxPair{});
+    return launch_pdl("col_absmax_kernel", col_absmax_kernel<__nv_bfloat16, false>, grid, dim3(kAbsmaxThreads), 0, st,
+                      1, static_cast<const uint8_t*>(x), rows, cols, per, absmax, (const float*)nullptr, AbsmaxPair{});
 }
 
 // Both calibrations of a layer in one launch: one wave of blocks shared between
@@ -862,12 +868,10 @@ sq_status calibrate_absmax_pair_impl(const void* x, int64_t T, const void* w, in
     pair.rc1 = (int)rc_x;
     const dim3 grid((unsigned)ct, (unsigned)(rc_x + rc_w));
     if (dt == SQ_F32)
-        col_absmax_kernel<float, false><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), T, K, per_x, xmax, nullptr, pair);
-    else
-        col_absmax_kernel<__nv_bfloat16, false><<<grid, kAbsmaxThreads, 0, st>>>(
-            static_cast<const uint8_t*>(x), T, K, per_x, xmax, nullptr, pair);
-    return check_launch("col_absmax_kernel<pair>");
+        return launch_pdl("col_absmax_kernel<pair>", col_absmax_kernel<float, false>, grid, dim3(kAbsmaxThreads), 0,
+                          st, 1, static_cast<const uint8_t*>(x), T, K, per_x, xmax, (const float*)nullptr, pair);
+    return launch_pdl("col_absmax_kernel<pair>", col_absmax_kernel<__nv_bfloat16, false>, grid, dim3(kAbsmaxThreads),
+                      0, st, 1, static_cast<const uint8_t*>(x), T, K, per_x, xmax, (const float*)nullptr, pair);
 }
 
 sq_status smooth_factors_impl(const float* xmax, const float* wmax, int64_t K, float alpha,
@@ -879,8 +883,8 @@ sq_status smooth_factors_impl(const float* xmax, const float* wmax, int64_t K, f
     if (!xmax || !wmax || !s) { set_error("NULL pointer"); return SQ_ERR_INVALID_ARG; }
     const int threads = 256;
     const int64_t blocks = (K + threads - 1) / threads;
-    smooth_factors_kernel<<<(unsigned)blocks, threads, 0, st>>>(xmax, wmax, K, alpha, eps, s);
-    return check_launch("smooth_factors_kernel");
+    return launch_pdl("smooth_factors_kernel", smooth_factors_kernel, dim3((unsigned)blocks), dim3(threads), 0, st, 1,
+                      xmax, wmax, K, alpha, eps, s);
 }
 
 static sq_status row_quant_common(int mode, const void* in, sq_dtype dt, int64_t rows, int64_t K,
