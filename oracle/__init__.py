@@ -109,6 +109,9 @@ def lib():
             L.sqo_quant_row_e4m3.argtypes = [vp, i64, vp, vp]
             L.sqo_quant_rows_e4m3_f64.argtypes = [vp, i64, i64, vp, vp]
             L.sqo_w8a8_e4m3_f64.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+            L.sqo_fold_quant_weights_e4m3.argtypes = [vp, ctypes.c_int, i64, i64, vp, vp, vp]
+            L.sqo_smooth_quant_act_e4m3.argtypes = [vp, ctypes.c_int, i64, i64, vp, vp, vp]
+            L.sqo_gemm_dequant_e4m3.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
             L.sqo_num_threads.restype = ctypes.c_int
             L.sqo_set_num_threads.argtypes = [ctypes.c_int]
             _lib = L
@@ -499,3 +502,37 @@ def w8a8_per_tensor_error_f64(X: np.ndarray, W: np.ndarray) -> float:
     Yq = np.empty((T, N), np.float64)
     lib().sqo_w8a8_f64(_p(xq.reshape(T, K)), _p(np.full(T, sa[0])), _p(wq), _p(sw), T, N, K, _p(Yq))
     return rel_frobenius_f64(Yq, matmul_xwT_f64(X, W))
+
+
+def fold_quant_weights_e4m3(w: np.ndarray, s: np.ndarray):
+    w = np.ascontiguousarray(w)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    N, K = w.shape
+    wq = np.empty((N, K), np.uint8)
+    ws = np.empty(N, np.float32)
+    lib().sqo_fold_quant_weights_e4m3(_p(w), _dt(w), N, K, _p(s), _p(wq), _p(ws))
+    return wq, ws
+
+
+def smooth_quant_act_e4m3(x: np.ndarray, s: np.ndarray):
+    x = np.ascontiguousarray(x)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    T, K = x.shape
+    xq = np.empty((T, K), np.uint8)
+    xs = np.empty(T, np.float32)
+    lib().sqo_smooth_quant_act_e4m3(_p(x), _dt(x), T, K, _p(s), _p(xq), _p(xs))
+    return xq, xs
+
+
+def gemm_dequant_e4m3(xq, x_scale, wq, w_scale):
+    """-> (y float32 [M, N], magnitude sum |products| * scales, fp64)."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    x_scale = np.ascontiguousarray(x_scale, dtype=np.float32)
+    w_scale = np.ascontiguousarray(w_scale, dtype=np.float32)
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = np.empty((M, N), np.float32)
+    mag = np.empty((M, N), np.float64)
+    lib().sqo_gemm_dequant_e4m3(_p(xq), _p(x_scale), _p(wq), _p(w_scale), M, N, K, _p(y), _p(mag))
+    return y, mag

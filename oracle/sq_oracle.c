@@ -713,6 +713,63 @@ void sqo_quant_row_e4m3(const float *v, int64_t K, uint8_t *q, float *scale_out)
     *scale_out = scale;
 }
 
+/* The FP8 path of the layer in fp32, in the order of the int8 path: weights
+ * folded (RN(W_nj s_j)) and activations smoothed (RN(X_tj / s_j)) exactly as
+ * in steps a3 and a4, then the per-row FP8 quantizer above. */
+void sqo_fold_quant_weights_e4m3(const void *w, int dt, int64_t N, int64_t K, const float *s,
+                                 uint8_t *wq, float *w_scale)
+{
+#pragma omp parallel
+    {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+#pragma omp for schedule(static)
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t j = 0; j < K; ++j) row[j] = load_elem(w, dt, n * K + j) * s[j];
+            sqo_quant_row_e4m3(row, K, wq + n * K, w_scale + n);
+        }
+        free(row);
+    }
+}
+
+void sqo_smooth_quant_act_e4m3(const void *x, int dt, int64_t T, int64_t K, const float *s,
+                               uint8_t *xq, float *x_scale)
+{
+#pragma omp parallel
+    {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            for (int64_t j = 0; j < K; ++j) row[j] = load_elem(x, dt, t * K + j) / s[j];
+            sqo_quant_row_e4m3(row, K, xq + t * K, x_scale + t);
+        }
+        free(row);
+    }
+}
+
+/* acc[t, n] = sum_k dec(xq[t,k]) dec(wq[n,k]) in fp64 (exact: every product of
+ * two E4M3 values has at most 8 significant bits between 2^-18 and 2^17.6, so
+ * sums of up to 32768 of them span fewer than 53 bits), then the epilogue of
+ * the int8 path on the sum rounded once to fp32:
+ *   y = (RN32(acc) * x_scale[t]) * w_scale[n]. mag (may be NULL) receives
+ * sum_k |dec(xq) dec(wq)| * x_scale * w_scale, the scale of accumulation error. */
+void sqo_gemm_dequant_e4m3(const uint8_t *xq, const float *x_scale, const uint8_t *wq, const float *w_scale,
+                           int64_t M, int64_t N, int64_t K, float *y, double *mag)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, am = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = sqo_e4m3_to_f64(xq[t * K + k]) * sqo_e4m3_to_f64(wq[n * K + k]);
+                acc += p;
+                am += fabs(p);
+            }
+            float v = ((float)acc * x_scale[t]) * w_scale[n];
+            y[t * N + n] = v;
+            if (mag) mag[t * N + n] = am * (double)x_scale[t] * (double)w_scale[n];
+        }
+}
+
 /* The same rule in fp64 for the error experiments. */
 void sqo_quant_rows_e4m3_f64(const double *v, int64_t rows, int64_t K, uint8_t *q, double *scale)
 {

@@ -457,6 +457,27 @@ def pin_e4m3_codes():
     assert _bits(sc) == _bits(rn32(Fraction(3) / 448)) and int(q[1]) == 0xFE
 
 
+
+def pin_e4m3_gemm_exact():
+    """FP8 product: codes decoded by torch.float8_e4m3fn (a library routine),
+    summed exactly in fp64 (numpy), rounded once to fp32, then (acc * sa) * sw
+    in fp32: equal to the oracle bit for bit."""
+    import torch
+    rng = np.random.default_rng(25)
+    M, N, K = 5, 7, 300
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    xq = rng.choice(codes, size=(M, K)).astype(np.uint8)
+    wq = rng.choice(codes, size=(N, K)).astype(np.uint8)
+    sa = rng.uniform(1e-3, 1.0, M).astype(np.float32)
+    sw = rng.uniform(1e-3, 1.0, N).astype(np.float32)
+    dx = torch.from_numpy(xq).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    dw = torch.from_numpy(wq).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    acc = dx @ dw.T
+    want = (acc.astype(np.float32) * sa[:, None]) * sw[None, :]
+    y, _ = oracle.gemm_dequant_e4m3(xq, sa, wq, sw)
+    assert np.array_equal(y.view(np.uint32), want.astype(np.float32).view(np.uint32))
+
+
 FAST_PINS = [
     pin_worked_example,
     pin_ties_half_even,
@@ -475,4 +496,5 @@ FAST_PINS = [
     pin_norm_fold,
     pin_decomposition_exact,
     pin_e4m3_codes,
+    pin_e4m3_gemm_exact,
 ]

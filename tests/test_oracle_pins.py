@@ -141,3 +141,20 @@ def test_alpha_search_fp32_path(experiment, oracle_lib):
     errs, best = oracle.alpha_search(X.astype(np.float32), W.astype(np.float32), alphas)
     assert [round(100 * e, 1) for e in errs] == [row["error_percent"] for row in g["alpha_table"]], errs
     assert best == 0.5
+
+
+def test_fp8_fp32_chain(experiment, oracle_lib):
+    """The fp32 FP8 path (folded / smoothed rows, per-row E4M3, exact sum, the
+    int8 path's epilogue) gives the printed 3.3% and 2.9% on the same data."""
+    g = pins.golden("format_and_granularity.json")
+    X, W, Y = experiment
+    X32, W32 = X.astype(np.float32), W.astype(np.float32)
+    errs = []
+    for s in (np.ones(X.shape[1], np.float32),
+              oracle.smooth_factors(oracle.col_absmax(X32), oracle.col_absmax(W32), 0.5)):
+        wq, sw = oracle.fold_quant_weights_e4m3(W32, s)
+        xq, sa = oracle.smooth_quant_act_e4m3(X32, s)
+        y, _ = oracle.gemm_dequant_e4m3(xq, sa, wq, sw)
+        errs.append(100 * oracle.rel_frobenius_f64(y.astype(np.float64), Y))
+    assert round(errs[0], 1) == g["per_token_fp8_percent_before"], errs
+    assert round(errs[1], 1) == g["per_token_fp8_percent_after"], errs
