@@ -219,6 +219,7 @@ VARIANTS = {
     "per_tensor_static": "a1(X) a1(W) a2 a3, static range from the calibration maxima, per-tensor codes, a5 (O3)",
     "rmsnorm": "a1(X) a1(W) a2 a3, gain fold, RMSNorm + per-token codes, a5 (the norm-folded O1)",
     "split": "a1(X), outlier split, bulk int8 of W and X, outlier gathers, int8 GEMM + fp32 outlier epilogue",
+    "fp8": "a1(X)+a1(W) in one launch, a2, a3 and a4 with FP8 E4M3 codes, the FP8 GEMM (fp32 accumulation)",
     "alpha_search": "one sq_alpha_search call: a1(X) a1(W), the float reference product, then per alpha "
                     "a2 a3 a4 a5 (fp32 out) and the error reduction",
 }
@@ -258,6 +259,23 @@ def build_step(variant, sq, wl, x, w, dev, stream):
         st.append(("alpha_search", search, once + len(alphas) * per_alpha, len(alphas) * ops))
         return maxima, st, {"alphas": alphas, "search": result,
                             "note": "the call synchronizes its stream; ops = int8 GEMM ops over all alphas"}
+    if variant == "fp8":
+        wq8 = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        xq8 = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        st.append(("a1_calibrate_xw", lambda: sq.sq_calibrate_absmax_pair(x, w, xmax, wmax, stream=stream),
+                   (M + N) * K * in_es + 2 * K * 4, 0))
+        st.append(("a2_smooth_factors", lambda: sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream),
+                   3 * K * 4, 0))
+        st.append(("a3_fold_quant_w_e4m3", lambda: sq.sq_fold_quant_weights_e4m3(w, s, wq=wq8, w_scale=wsc,
+                                                                               stream=stream),
+                   N * K * in_es + K * 4 + N * K + N * 4, 0))
+        st.append(("a4_smooth_quant_x_e4m3", lambda: sq.sq_smooth_quant_act_e4m3(x, s, xq=xq8, x_scale=xsc,
+                                                                                 stream=stream),
+                   M * K * in_es + K * 4 + M * K + M * 4, 0))
+        st.append(("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm_e4m3(xq8, xsc, wq8, wsc, y=y, stream=stream),
+                   gemm_bytes, ops))
+        return maxima, st, {"note": "FP8 E4M3 codes; the GEMM kernel is the paired-SM tcgen05 kernel with "
+                                    "kind::f8f6f4 operands"}
     if variant == "smoothquant":
         st.append(("a1_calibrate_xw", lambda: sq.sq_calibrate_absmax_pair(x, w, xmax, wmax, stream=stream),
                    (M + N) * K * in_es + 2 * K * 4, 0))
@@ -447,11 +465,12 @@ def run_ours(args, world, rank, local):
     if args.variant == "alpha_search":
         pass
     elif M > 16:
-        roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel (a5, paired-SM tcgen05)" if M > 128
-                    else "gemm_tiled_kernel (a5)",
+        roofline = {"bound": "tensor", "kernel": ("gemm_pair_kernel (a5, paired-SM tcgen05)" if M > 128
+                                                  else "gemm_tiled_kernel (a5)")
+                    + (", FP8 E4M3 operands" if args.variant == "fp8" else ""),
                     "achieved": round(achieved, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
                     "frac": round(achieved / int8_peak, 4),
-                    "traffic": load_traffic() if (M > 128 and default_gemm) else None,
+                    "traffic": load_traffic() if (M > 128 and default_gemm and args.variant != "fp8") else None,
                     "peak_source": f"{peak_src}: bf16 {bf16_peak} TFLOP/s (burst) x {INT8_OVER_BF16} nominal "
                                    f"int8/bf16 ratio",
                     "algorithmic_ops_per_launch": ops}

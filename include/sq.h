@@ -328,6 +328,32 @@ sq_status sq_alpha_search(const void* x, const void* w, sq_dtype in_dt, int64_t 
                           double* err, float* best_alpha, void* workspace, size_t ws_bytes,
                           sq_stream_t stream);
 
+/* ---------------------------------------------------------------- FP8 E4M3 sibling
+ * The same layer with FP8 E4M3 codes instead of int8: per-token activation
+ * scales and per-output-channel weight scales amax / 448, each quotient
+ * converted to E4M3 with round-to-nearest-even and saturation to +-448 (the
+ * format has no infinities), and the GEMM on the FP8 tensor cores with fp32
+ * accumulation ("Why do activation outliers break INT8 W8A8...", "A strong
+ * answer": per-token FP8 activations keep about 3 mantissa bits of relative
+ * precision for small values, so smoothing matters less: 3.3% error before
+ * smoothing, 2.9% after, on the page's synthetic data).
+ *
+ * sq_fold_quant_weights_e4m3 / sq_smooth_quant_act_e4m3: as
+ *   sq_fold_quant_weights / sq_smooth_quant_act (same fold and smoothing, fp32
+ *   division for the quotient), codes are E4M3 bytes, scale = amax / 448 (1.0
+ *   for an all-zero row). K <= 65536.
+ * sq_w8a8_gemm_e4m3: acc_tn = sum_k dec(xq_tk) dec(wq_nk) accumulated by the
+ *   tensor cores in fp32 (every product of two E4M3 values is exact in fp32;
+ *   the order of the additions is the hardware's), y_tn = (acc_tn * x_scale_t)
+ *   * w_scale_n, out_dt SQ_F32 or SQ_BF16. No workspace. */
+sq_status sq_fold_quant_weights_e4m3(const void* w, sq_dtype dt, int64_t N, int64_t K, const float* s,
+                                     uint8_t* wq, float* w_scale, sq_stream_t stream);
+sq_status sq_smooth_quant_act_e4m3(const void* x, sq_dtype dt, int64_t T, int64_t K, const float* s,
+                                   uint8_t* xq, float* x_scale, sq_stream_t stream);
+sq_status sq_w8a8_gemm_e4m3(const uint8_t* xq, const float* x_scale, const uint8_t* wq,
+                            const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
+                            sq_dtype out_dt, sq_stream_t stream);
+
 /* ---------------------------------------------------------------- whole layer
  * The whole path on one batch: calibrate X and W (a1, from zero), smoothing
  * factors (a2), fold + quantize W (a3), smooth + quantize X (a4), GEMM with

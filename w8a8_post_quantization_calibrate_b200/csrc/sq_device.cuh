@@ -144,6 +144,16 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t
                  : "memory");
 }
 
+// The same for FP8: kind::f8f6f4 with E4M3 A and B (both operands one type), fp32 D.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -171,6 +181,16 @@ __host__ __device__ constexpr uint32_t make_idesc_i8(int M, int N) {
     return (2u << 4)                          // D format: s32
          | (1u << 7)                          // A format: signed 8-bit
          | (1u << 10)                         // B format: signed 8-bit
+         | ((uint32_t)(N >> 3) << 17)         // N / 8
+         | ((uint32_t)(M >> 4) << 24);        // M / 16
+}
+
+// Instruction descriptor, kind::f8f6f4: E4M3 A and B (format code 0), fp32 D
+// (format code 1), both operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N) {
+    return (1u << 4)                          // D format: f32
+         | (0u << 7)                          // A format: E4M3
+         | (0u << 10)                         // B format: E4M3
          | ((uint32_t)(N >> 3) << 17)         // N / 8
          | ((uint32_t)(M >> 4) << 24);        // M / 16
 }
@@ -210,6 +230,12 @@ __device__ __forceinline__ void tmem_wait_ld() {
 // (explicit intrinsics: never contracted into an FMA).
 __device__ __forceinline__ float dequant(int32_t acc, float sa, float sw) {
     return __fmul_rn(__fmul_rn(__int2float_rn(acc), sa), sw);
+}
+// The epilogue value of a raw 32-bit accumulator: int32 (int8 operands) or fp32 (FP8).
+template <bool F8>
+__device__ __forceinline__ float dequant_raw(uint32_t acc, float sa, float sw) {
+    if (F8) return __fmul_rn(__fmul_rn(__uint_as_float(acc), sa), sw);
+    return dequant((int32_t)acc, sa, sw);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -49,6 +49,7 @@ constexpr int ACC_COLS = BN;                    // int32 columns per accumulator
 constexpr int TMEM_COLS = 2 * ACC_COLS;         // double-buffered: 512 columns
 constexpr int GEMM_THREADS = 192;               // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint32_t IDESC_TILED = make_idesc_i8(BM, BN);
+constexpr uint32_t IDESC_TILED_E4M3 = make_idesc_e4m3(BM, BN);
 
 constexpr int S_BM = 128;        // weight rows per tile (MMA M)
 constexpr int S_BN = 16;         // tokens (MMA N)
@@ -68,6 +69,13 @@ constexpr size_t tiled_smem_bytes() {
 }
 constexpr size_t stream_smem_bytes() {
     return 1024 + S_STAGES * (S_A_STAGE + S_B_STAGE) + 256;
+}
+
+// One MMA of the 1-CTA kernel: int8 or FP8 E4M3 operands.
+template <bool F8>
+__device__ __forceinline__ void mma_tiled(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    if (F8) mma_f8(d_tmem, adesc, bdesc, IDESC_TILED_E4M3, accumulate);
+    else mma_i8(d_tmem, adesc, bdesc, IDESC_TILED, accumulate);
 }
 
 // Tile order: groups of 16 row tiles, column tiles outermost inside a group, so
@@ -160,7 +168,7 @@ __device__ __forceinline__ float add_split1(float v, int64_t t, int64_t n, const
 }
 
 // Stores 32 consecutive outputs of one row (row-major y, row stride N).
-template <int OUT, bool SPLIT>
+template <int OUT, bool SPLIT, bool F8 = false>
 __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int N, const uint32_t (&r)[32],
                                             float sa, const float* __restrict__ w_scale, const float* xr,
                                             const float* ws_col, int ld) {
@@ -183,15 +191,15 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
             const float4 sw = __ldg(reinterpret_cast<const float4*>(w_scale + col0 + i));
-            v[i] = dequant((int32_t)r[i], sa, sw.x);
-            v[i + 1] = dequant((int32_t)r[i + 1], sa, sw.y);
-            v[i + 2] = dequant((int32_t)r[i + 2], sa, sw.z);
-            v[i + 3] = dequant((int32_t)r[i + 3], sa, sw.w);
+            v[i] = dequant_raw<F8>(r[i], sa, sw.x);
+            v[i + 1] = dequant_raw<F8>(r[i + 1], sa, sw.y);
+            v[i + 2] = dequant_raw<F8>(r[i + 2], sa, sw.z);
+            v[i + 3] = dequant_raw<F8>(r[i + 3], sa, sw.w);
         }
     } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-            v[i] = (col0 + i < N) ? dequant((int32_t)r[i], sa, __ldg(w_scale + col0 + i)) : 0.0f;
+            v[i] = (col0 + i < N) ? dequant_raw<F8>(r[i], sa, __ldg(w_scale + col0 + i)) : 0.0f;
     }
     if (SPLIT) add_split32(v, xr, ws_col, ld);
     if (OUT == kOutF32) {
@@ -224,7 +232,7 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
 }
 
 // ================================================================== prefill
-template <int OUT, bool SPLIT>
+template <int OUT, bool SPLIT, bool F8 = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const float* __restrict__ x_scale, const float* __restrict__ w_scale,
@@ -334,8 +342,8 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k)
-                        mma_i8(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
-                               make_sw128_kmajor_desc(b0 + k * UMMA_K), IDESC_TILED,
+                        mma_tiled<F8>(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
+                               make_sw128_kmajor_desc(b0 + k * UMMA_K),
                                (kb | k) != 0 ? 1u : 0u);
                     mma_commit(bar(EMPTY + stage));
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -376,9 +384,9 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 const int col0 = nb * BN + c * 32;
                 const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
                 if (row_ok && col0 < N)
-                    store_row32<OUT, SPLIT>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
+                    store_row32<OUT, SPLIT, F8>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
                 if (row_ok && col0 + 32 < N)
-                    store_row32<OUT, SPLIT>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
+                    store_row32<OUT, SPLIT, F8>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
             }
             tc_fence_before();
             __syncwarp();
@@ -440,6 +448,21 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uin
                  "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}"
                  :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+constexpr uint32_t IDESC_PAIR_E4M3 = make_idesc_e4m3(256, 256);
+// One MMA of the pair: int8 or FP8 E4M3 operands.
+template <bool F8>
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    if (F8) mma_f8_pair(d_tmem, adesc, bdesc, IDESC_PAIR_E4M3, accumulate);
+    else mma_i8_pair(d_tmem, adesc, bdesc, IDESC_PAIR, accumulate);
+}
+
 // Arrive once on `bar` in both CTAs of the pair when the MMAs issued so far are done.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
@@ -473,7 +496,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "n"(NCOLS) : "memory");
 }
 
-template <int OUT, bool SPLIT>
+template <int OUT, bool SPLIT, bool F8 = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ x_scale, const float* __restrict__ w_scale,
@@ -596,8 +619,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const uint32_t b0 = smem_u32(sB + stage * P_B_STAGE);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k)
-                        mma_i8_pair(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
-                                    make_sw128_kmajor_desc(b0 + k * UMMA_K), IDESC_PAIR, (kb | k) != 0 ? 1u : 0u);
+                        mma_pair<F8>(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
+                                     make_sw128_kmajor_desc(b0 + k * UMMA_K), (kb | k) != 0 ? 1u : 0u);
                     mma_commit_pair(bar(EMPTY + stage));
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -636,9 +659,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const int col0 = nb * BN + c * 32;
                 const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
                 if (row_ok && col0 < N)
-                    store_row32<OUT, SPLIT>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
+                    store_row32<OUT, SPLIT, F8>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
                 if (row_ok && col0 + 32 < N)
-                    store_row32<OUT, SPLIT>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
+                    store_row32<OUT, SPLIT, F8>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
             }
             tc_fence_before();
             __syncwarp();
@@ -923,32 +946,32 @@ sq_status ensure_smem_attr(Kern k, size_t bytes, bool& done) {
     return SQ_OK;
 }
 
-template <int OUT, bool SPLIT = false>
+template <int OUT, bool SPLIT = false, bool F8 = false>
 sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
                        int M, int N, int K, cudaStream_t st, const SplitTerm& sp = SplitTerm{}) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const size_t smem = tiled_smem_bytes() + (SPLIT ? kSplitSmem : 0);
-    sq_status r = ensure_smem_attr(gemm_tiled_kernel<OUT, SPLIT>, smem, attr_done[di.device & 63]);
+    sq_status r = ensure_smem_attr(gemm_tiled_kernel<OUT, SPLIT, F8>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = tiles < di.sm_count ? tiles : di.sm_count;
-    return launch_pdl("gemm_tiled_kernel", gemm_tiled_kernel<OUT, SPLIT>, dim3(grid), dim3(GEMM_THREADS), smem, st, 1,
+    return launch_pdl("gemm_tiled_kernel", gemm_tiled_kernel<OUT, SPLIT, F8>, dim3(grid), dim3(GEMM_THREADS), smem, st, 1,
                       ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
 }
 
-template <int OUT, bool SPLIT = false>
+template <int OUT, bool SPLIT = false, bool F8 = false>
 sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
                       int M, int N, int K, cudaStream_t st, const SplitTerm& sp = SplitTerm{}) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const size_t smem = pair_smem_bytes() + (SPLIT ? kSplitSmem : 0);
-    sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT, SPLIT>, smem, attr_done[di.device & 63]);
+    sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT, SPLIT, F8>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const int tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int max_pairs = di.sm_count / 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
-    return launch_pdl("gemm_pair_kernel", gemm_pair_kernel<OUT, SPLIT>, dim3(2 * pairs), dim3(GEMM_THREADS), smem, st,
+    return launch_pdl("gemm_pair_kernel", gemm_pair_kernel<OUT, SPLIT, F8>, dim3(2 * pairs), dim3(GEMM_THREADS), smem, st,
                       2, ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
 }
 
@@ -1058,6 +1081,38 @@ sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq
     }
 }
 
+// FP8 E4M3 operands, fp32 accumulation in TMEM: the paired-SM kernel for
+// M > 128, the 1-CTA kernel otherwise (no split-K path: fp32 partial sums
+// merged by atomics would depend on their order).
+sq_status gemm_e4m3_impl(const uint8_t* xq, const float* x_scale, const uint8_t* wq, const float* w_scale, int64_t M,
+                         int64_t N, int64_t K, void* y, sq_dtype out_dt, cudaStream_t st) {
+    if (M < 0 || N < 0 || K < 0) { set_error("negative size"); return SQ_ERR_INVALID_ARG; }
+    if (out_dt != SQ_F32 && out_dt != SQ_BF16) { set_error("output dtype must be SQ_F32 or SQ_BF16"); return SQ_ERR_UNSUPPORTED; }
+    if (M == 0 || N == 0) return SQ_OK;
+    if (K == 0 || K % 16 != 0) { set_error("K=%lld must be a positive multiple of 16", (long long)K); return SQ_ERR_UNSUPPORTED; }
+    if (M > 2147483647LL || N > 2147483647LL || K > 2147483647LL) { set_error("size too large"); return SQ_ERR_UNSUPPORTED; }
+    if (!xq || !wq || !y || !x_scale || !w_scale) { set_error("NULL pointer"); return SQ_ERR_INVALID_ARG; }
+    if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || !aligned16(w_scale)) {
+        set_error("xq, wq, y and w_scale must be 16-byte aligned");
+        return SQ_ERR_UNSUPPORTED;
+    }
+    sq_status r;
+    CUtensorMap ta, tb;
+    const SplitTerm none;
+    if (M > 128) {
+        if ((r = make_map_i8(&ta, xq, M, K, 128)) != SQ_OK) return r;
+        if ((r = make_map_i8(&tb, wq, N, K, 128)) != SQ_OK) return r;
+        return out_dt == SQ_F32
+            ? launch_pair<kOutF32, false, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, none)
+            : launch_pair<kOutBF16, false, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, none);
+    }
+    if ((r = make_map_i8(&ta, xq, M, K, BM)) != SQ_OK) return r;
+    if ((r = make_map_i8(&tb, wq, N, K, BN)) != SQ_OK) return r;
+    return out_dt == SQ_F32
+        ? launch_tiled<kOutF32, false, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, none)
+        : launch_tiled<kOutBF16, false, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, none);
+}
+
 sq_status gemm_split_impl(const int8_t* xq, const float* x_scale, const int8_t* wq, const float* w_scale,
                           int64_t M, int64_t N, int64_t K, const float* x_out, const float* w_out, int64_t ld,
                           void* y, sq_dtype out_dt, void* workspace, size_t ws_bytes, cudaStream_t st) {
@@ -1096,6 +1151,11 @@ sq_status sq_w8a8_gemm(const int8_t* xq, const float* x_scale, const int8_t* wq,
                        size_t ws_bytes, sq_stream_t stream) {
     return sq::gemm_dispatch(xq, x_scale, wq, w_scale, M, N, K, y, out_dt, workspace, ws_bytes,
                              (cudaStream_t)stream, nullptr);
+}
+
+sq_status sq_w8a8_gemm_e4m3(const uint8_t* xq, const float* x_scale, const uint8_t* wq, const float* w_scale,
+                            int64_t M, int64_t N, int64_t K, void* y, sq_dtype out_dt, sq_stream_t stream) {
+    return sq::gemm_e4m3_impl(xq, x_scale, wq, w_scale, M, N, K, y, out_dt, (cudaStream_t)stream);
 }
 
 sq_status sq_w8a8_gemm_split(const int8_t* xq, const float* x_scale, const int8_t* wq, const float* w_scale,

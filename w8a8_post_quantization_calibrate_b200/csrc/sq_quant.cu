@@ -10,6 +10,7 @@
 // __fdiv_rn, never contracted), rounding to nearest-even, so the codes and
 // scales are reproducible bit for bit on any IEEE implementation.
 #include <cstdio>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "sq_device.cuh"
@@ -195,13 +196,21 @@ struct Chunk8<__nv_bfloat16> {
     }
 };
 
+// Code formats of the row quantizer: symmetric int8 ([-127, 127], scale =
+// amax / 127) or FP8 E4M3 (scale = amax / 448, the quotient converted with
+// round-to-nearest-even and saturation to +-448).
+enum CodeFormat { kInt8 = 0, kE4M3 = 1 };
+
+template <int FMT>
 __device__ __forceinline__ uint32_t code8(float v, float scale) {
+    if (FMT == kE4M3)
+        return (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v, scale), __NV_SATFINITE, __NV_E4M3);
     int q = __float2int_rn(__fdiv_rn(v, scale));
     q = max(-127, min(127, q));
     return static_cast<uint32_t>(q) & 0xffu;
 }
 
-template <typename T, int MODE, int TPB, int MAXC>
+template <typename T, int MODE, int TPB, int MAXC, int FMT>
 __global__ void __launch_bounds__(TPB)
 row_quant_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
                  int8_t* __restrict__ q, float* __restrict__ scale_out) {
@@ -242,7 +251,7 @@ row_quant_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float*
         for (int w = 1; w < NW; ++w) amax = fmaxf(amax, red[parity][w]);
 
         const bool zero = (amax == 0.0f);
-        const float scale = zero ? 1.0f : __fdiv_rn(amax, 127.0f);
+        const float scale = zero ? 1.0f : __fdiv_rn(amax, FMT == kE4M3 ? 448.0f : 127.0f);
         int8_t* rq = q + row * K;
 #pragma unroll
         for (int i = 0; i < MAXC; ++i) {
@@ -250,10 +259,10 @@ row_quant_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float*
             if (c < nchunks) {
                 uint2 packed = make_uint2(0u, 0u);
                 if (!zero) {
-                    packed.x = code8(v[i][0], scale) | (code8(v[i][1], scale) << 8) |
-                               (code8(v[i][2], scale) << 16) | (code8(v[i][3], scale) << 24);
-                    packed.y = code8(v[i][4], scale) | (code8(v[i][5], scale) << 8) |
-                               (code8(v[i][6], scale) << 16) | (code8(v[i][7], scale) << 24);
+                    packed.x = code8<FMT>(v[i][0], scale) | (code8<FMT>(v[i][1], scale) << 8) |
+                               (code8<FMT>(v[i][2], scale) << 16) | (code8<FMT>(v[i][3], scale) << 24);
+                    packed.y = code8<FMT>(v[i][4], scale) | (code8<FMT>(v[i][5], scale) << 8) |
+                               (code8<FMT>(v[i][6], scale) << 16) | (code8<FMT>(v[i][7], scale) << 24);
                 }
                 *reinterpret_cast<uint2*>(rq + c * 8) = packed;
             }
@@ -656,23 +665,23 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
 // ============================================================== host side
 namespace {
 
-template <typename T, int MODE, int TPB, int MAXC>
+template <typename T, int MODE, int TPB, int MAXC, int FMT>
 sq_status launch_row_quant_inst(const void* in, int64_t rows, int64_t K, const float* s,
                                 int8_t* q, float* scale, cudaStream_t st) {
     const int64_t max_blocks = (int64_t)device_info().sm_count * (2048 / TPB);
     const int grid = (int)(rows < max_blocks ? rows : max_blocks);
-    return launch_pdl("row_quant_kernel", row_quant_kernel<T, MODE, TPB, MAXC>, dim3(grid), dim3(TPB), 0, st, 1,
+    return launch_pdl("row_quant_kernel", row_quant_kernel<T, MODE, TPB, MAXC, FMT>, dim3(grid), dim3(TPB), 0, st, 1,
                       static_cast<const T*>(in), rows, K, s, q, scale);
 }
 
-template <typename T, int MODE, int TPB>
+template <typename T, int MODE, int TPB, int FMT>
 sq_status launch_row_quant_tpb(int maxc, const void* in, int64_t rows, int64_t K, const float* s,
                                int8_t* q, float* scale, cudaStream_t st) {
     switch (maxc) {
-        case 1: return launch_row_quant_inst<T, MODE, TPB, 1>(in, rows, K, s, q, scale, st);
-        case 2: return launch_row_quant_inst<T, MODE, TPB, 2>(in, rows, K, s, q, scale, st);
-        case 4: return launch_row_quant_inst<T, MODE, TPB, 4>(in, rows, K, s, q, scale, st);
-        case 8: return launch_row_quant_inst<T, MODE, TPB, 8>(in, rows, K, s, q, scale, st);
+        case 1: return launch_row_quant_inst<T, MODE, TPB, 1, FMT>(in, rows, K, s, q, scale, st);
+        case 2: return launch_row_quant_inst<T, MODE, TPB, 2, FMT>(in, rows, K, s, q, scale, st);
+        case 4: return launch_row_quant_inst<T, MODE, TPB, 4, FMT>(in, rows, K, s, q, scale, st);
+        case 8: return launch_row_quant_inst<T, MODE, TPB, 8, FMT>(in, rows, K, s, q, scale, st);
     }
     set_error("internal: unsupported chunk count %d", maxc);
     return SQ_ERR_UNSUPPORTED;
@@ -682,6 +691,28 @@ int pow2ceil(int64_t v) {
     int p = 1;
     while (p < v) p <<= 1;
     return p;
+}
+
+// The IEEE-division kernel: one CTA per row at a time, K up to 65536.
+template <typename T, int MODE, int FMT>
+sq_status launch_row_quant_exact(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q, float* scale,
+                                 cudaStream_t st) {
+    const int64_t nchunks = K / 8;
+    int64_t tpb = pow2ceil((nchunks + 3) / 4);
+    if (tpb < 128) tpb = 128;
+    if (tpb > 1024) tpb = 1024;
+    const int64_t per = (nchunks + tpb - 1) / tpb;
+    const int maxc = pow2ceil(per);
+    if (maxc > 8) {
+        set_error("K=%lld exceeds the row-quantization limit of 65536", (long long)K);
+        return SQ_ERR_UNSUPPORTED;
+    }
+    switch (tpb) {
+        case 128: return launch_row_quant_tpb<T, MODE, 128, FMT>(maxc, in, rows, K, s, q, scale, st);
+        case 256: return launch_row_quant_tpb<T, MODE, 256, FMT>(maxc, in, rows, K, s, q, scale, st);
+        case 512: return launch_row_quant_tpb<T, MODE, 512, FMT>(maxc, in, rows, K, s, q, scale, st);
+        default: return launch_row_quant_tpb<T, MODE, 1024, FMT>(maxc, in, rows, K, s, q, scale, st);
+    }
 }
 
 template <typename T, int MODE, int R>
@@ -735,22 +766,7 @@ sq_status launch_row_quant(const void* in, int64_t rows, int64_t K, const float*
                   (long long)(32 * 16 * 8 * RowFastCPL<T>::value));
         return SQ_ERR_UNSUPPORTED;
     } else {
-    // longer rows: the IEEE-division kernel
-    int64_t tpb = pow2ceil((nchunks + 3) / 4);
-    if (tpb < 128) tpb = 128;
-    if (tpb > 1024) tpb = 1024;
-    const int64_t per = (nchunks + tpb - 1) / tpb;
-    const int maxc = pow2ceil(per);
-    if (maxc > 8) {
-        set_error("K=%lld exceeds the row-quantization limit of 65536", (long long)K);
-        return SQ_ERR_UNSUPPORTED;
-    }
-    switch (tpb) {
-        case 128: return launch_row_quant_tpb<T, MODE, 128>(maxc, in, rows, K, s, q, scale, st);
-        case 256: return launch_row_quant_tpb<T, MODE, 256>(maxc, in, rows, K, s, q, scale, st);
-        case 512: return launch_row_quant_tpb<T, MODE, 512>(maxc, in, rows, K, s, q, scale, st);
-        default: return launch_row_quant_tpb<T, MODE, 1024>(maxc, in, rows, K, s, q, scale, st);
-    }
+    return launch_row_quant_exact<T, MODE, kInt8>(in, rows, K, s, q, scale, st);
     }
 }
 
@@ -903,6 +919,25 @@ static sq_status row_quant_common(int mode, const void* in, sq_dtype dt, int64_t
                         : launch_row_quant<__nv_bfloat16, kSmooth>(in, rows, K, s, q, scale, st);
 }
 
+// FP8 E4M3 codes: the same fold / smoothing, per-row scale amax / 448, every
+// quotient an IEEE division (the exact kernel).
+static sq_status row_quant_e4m3_common(int mode, const void* in, sq_dtype dt, int64_t rows, int64_t K,
+                                       const float* s, uint8_t* q, float* scale, cudaStream_t st) {
+    sq_status r;
+    if ((r = check_input_dtype(dt)) != SQ_OK) return r;
+    if ((r = check_matrix(in, rows, K, "input")) != SQ_OK) return r;
+    if (rows == 0) return SQ_OK;
+    if (K == 0) { set_error("K must be positive"); return SQ_ERR_INVALID_ARG; }
+    if (!s || !q || !scale) { set_error("NULL pointer"); return SQ_ERR_INVALID_ARG; }
+    if (!aligned16(s) || !aligned16(q)) { set_error("s and codes must be 16-byte aligned"); return SQ_ERR_UNSUPPORTED; }
+    int8_t* qq = reinterpret_cast<int8_t*>(q);
+    if (mode == kFold)
+        return dt == SQ_F32 ? launch_row_quant_exact<float, kFold, kE4M3>(in, rows, K, s, qq, scale, st)
+                            : launch_row_quant_exact<__nv_bfloat16, kFold, kE4M3>(in, rows, K, s, qq, scale, st);
+    return dt == SQ_F32 ? launch_row_quant_exact<float, kSmooth, kE4M3>(in, rows, K, s, qq, scale, st)
+                        : launch_row_quant_exact<__nv_bfloat16, kSmooth, kE4M3>(in, rows, K, s, qq, scale, st);
+}
+
 sq_status fold_quant_weights_impl(const void* w, sq_dtype dt, int64_t N, int64_t K, const float* s,
                                   int8_t* wq, float* w_scale, cudaStream_t st) {
     return row_quant_common(kFold, w, dt, N, K, s, wq, w_scale, st);
@@ -916,6 +951,17 @@ sq_status smooth_quant_act_impl(const void* x, sq_dtype dt, int64_t T, int64_t K
 }  // namespace sq
 
 extern "C" {
+
+sq_status sq_fold_quant_weights_e4m3(const void* w, sq_dtype dt, int64_t N, int64_t K, const float* s, uint8_t* wq,
+                                     float* w_scale, sq_stream_t stream) {
+    return sq::row_quant_e4m3_common(sq::kFold, w, dt, N, K, s, wq, w_scale, (cudaStream_t)stream);
+}
+
+sq_status sq_smooth_quant_act_e4m3(const void* x, sq_dtype dt, int64_t T, int64_t K, const float* s, uint8_t* xq,
+                                   float* x_scale, sq_stream_t stream) {
+    return sq::row_quant_e4m3_common(sq::kSmooth, x, dt, T, K, s, xq, x_scale, (cudaStream_t)stream);
+}
+
 
 sq_status sq_calibrate_absmax_pair(const void* x, int64_t T, const void* w, int64_t N, sq_dtype dt, int64_t K,
                                    float* xmax, float* wmax, sq_stream_t stream) {

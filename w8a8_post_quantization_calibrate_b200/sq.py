@@ -44,6 +44,9 @@ _SIGS = {
     "sq_fold_quant_weights": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_smooth_quant_act": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_calibrate_absmax_pair": ([_vp, _i64, _vp, _i64, _int, _i64, _vp, _vp, _vp], _int),
+    "sq_fold_quant_weights_e4m3": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "sq_smooth_quant_act_e4m3": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
+    "sq_w8a8_gemm_e4m3": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp], _int),
     "sq_tensor_absmax": ([_vp, _int, _i64, _i64, _vp, _vp, _vp], _int),
     "sq_quant_act_per_tensor": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp], _int),
     "sq_fold_norm_gain": ([_vp, _int, _i64, _vp, _vp, _vp], _int),
@@ -172,6 +175,41 @@ def sq_calibrate_absmax_pair(x: torch.Tensor, w: torch.Tensor, xmax: torch.Tenso
     _check(_lib.sq_calibrate_absmax_pair(_dev(x, "x"), T, _dev(w, "w"), N, _dt(x), K, _dev(xmax, "xmax"),
                                          _dev(wmax, "wmax"), _stream(stream)), "sq_calibrate_absmax_pair")
     return xmax, wmax
+
+
+def sq_fold_quant_weights_e4m3(w: torch.Tensor, s: torch.Tensor, wq=None, w_scale=None, stream=None):
+    """Fold s into W, per-output-channel FP8 E4M3 -> (codes uint8 [N, K], w_scale)."""
+    N, K = w.shape
+    if wq is None:
+        wq = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=w.device)
+    _check(_lib.sq_fold_quant_weights_e4m3(_dev(w, "w"), _dt(w), N, K, _dev(s, "s"), _dev(wq, "wq"),
+                                           _dev(w_scale, "w_scale"), _stream(stream)), "sq_fold_quant_weights_e4m3")
+    return wq, w_scale
+
+
+def sq_smooth_quant_act_e4m3(x: torch.Tensor, s: torch.Tensor, xq=None, x_scale=None, stream=None):
+    """Smooth X by s, per-token FP8 E4M3 -> (codes uint8 [T, K], x_scale)."""
+    T, K = x.shape
+    if xq is None:
+        xq = torch.empty((T, K), dtype=torch.uint8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(_lib.sq_smooth_quant_act_e4m3(_dev(x, "x"), _dt(x), T, K, _dev(s, "s"), _dev(xq, "xq"),
+                                         _dev(x_scale, "x_scale"), _stream(stream)), "sq_smooth_quant_act_e4m3")
+    return xq, x_scale
+
+
+def sq_w8a8_gemm_e4m3(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                      out_dtype=torch.bfloat16, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    M, K = xq.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    _check(_lib.sq_w8a8_gemm_e4m3(_dev(xq, "xq"), _dev(x_scale, "x_scale"), _dev(wq, "wq"), _dev(w_scale, "w_scale"),
+                                  M, N, K, _dev(y, "y"), _dt(y), _stream(stream)), "sq_w8a8_gemm_e4m3")
+    return y
 
 
 def _opt_dev(t: torch.Tensor | None, name: str):
