@@ -50,7 +50,8 @@ struct Vec16<__nv_bfloat16> {
 };
 
 constexpr int kAbsmaxThreads = 256;
-constexpr int kAbsmaxRowsInFlight = 8;   // per warp; a block covers 64 rows per iteration
+constexpr int kAbsmaxRowsInFlight = 8;   // per warp (two batches); blocks cover multiples of 64 rows
+constexpr int kAbsmaxBatch = 4;          // rows per warp per batch
 
 // Two tensors in one launch (the activations and the weights of a layer share
 // K): row-chunk blocks [0, rc1) read the first, the others the second.
@@ -94,16 +95,29 @@ col_absmax_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t cols,
 
     if (col < cols) {
         const uint8_t* p = x + col * (int64_t)sizeof(T);
-        // 8 rows per warp in flight: all loads are issued before any is used.
-        for (int64_t r = r_begin + warp; r < r_end; r += 8 * kAbsmaxRowsInFlight) {
-            uint4 v[kAbsmaxRowsInFlight];
+        // Batches of kAbsmaxBatch rows per warp, double-buffered: the next
+        // batch's loads are issued before the current one is reduced, so a
+        // warp always has rows in flight.
+        constexpr int B = kAbsmaxBatch;
+        constexpr int64_t step = 8 * B;
+        uint4 cur[B], nxt[B];
+        int64_t r = r_begin + warp;
 #pragma unroll
-            for (int u = 0; u < kAbsmaxRowsInFlight; ++u) {
-                const int64_t rr = r + 8 * u;
-                v[u] = rr < r_end ? ld_stream_v4(p + rr * row_bytes) : make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < B; ++u) {
+            const int64_t rr = r + 8 * u;
+            cur[u] = rr < r_end ? ld_stream_v4(p + rr * row_bytes) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (; r < r_end; r += step) {
+            const int64_t rn = r + step;
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                const int64_t rr = rn + 8 * u;
+                nxt[u] = rr < r_end ? ld_stream_v4(p + rr * row_bytes) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
-            for (int u = 0; u < kAbsmaxRowsInFlight; ++u) Vec16<T>::absmax(m, v[u]);
+            for (int u = 0; u < B; ++u) Vec16<T>::absmax(m, cur[u]);
+#pragma unroll
+            for (int u = 0; u < B; ++u) cur[u] = nxt[u];
         }
     }
 
