@@ -362,8 +362,13 @@ sq_status sq_w8a8_gemm_e4m3(const uint8_t* xq, const float* x_scale, const uint8
  *   y [M x N]: dtype out_dt (SQ_F32 or SQ_BF16).
  *   x, w and y may each be device memory or host memory (pinned host memory
  *   copies asynchronously; pageable host memory makes the copy synchronous).
- *   Host operands are staged through the workspace with cudaMemcpyAsync on
- *   `stream`; for a host y the call returns before the copy-back completes, so
+ *   Host x and w are staged through the workspace by a copy stream of the
+ *   library, so that one call's input copies overlap the previous call's GEMM
+ *   and output copy: they wait only until the previous call through the same
+ *   workspace has finished reading its staged inputs, not for other work
+ *   enqueued earlier on `stream` -- the host buffers must hold the inputs when
+ *   the call is made. The kernels run on `stream` after those copies. A host y
+ *   is copied back on `stream`; the call returns before the copy completes, so
  *   synchronize `stream` before reading it.
  *   workspace: device, ws_bytes >= sq_linear_workspace_size(...); it holds the
  *   maxima, factors, codes, scales and (for host operands) the staged copies.

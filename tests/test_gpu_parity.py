@@ -372,6 +372,27 @@ def test_sq_linear_matches_steps_device_and_host():
     assert_f32_close(yh.numpy(), ref["y"], "sq_linear host")
 
 
+def test_sq_linear_back_to_back_host_calls():
+    """Host operands through one workspace, three calls without a sync in
+    between (each call's input copies overlap the previous call's GEMM and
+    output copy): every output equals the oracle's."""
+    wl = synth.WORKLOADS["tiny"]
+    outs, refs = [], []
+    ws = torch.zeros(sq.sq_linear_workspace_size(200, 300, 1024, torch.float32, torch.float32),
+                     dtype=torch.uint8, device=DEV)
+    for i in range(3):
+        x, w = synth.make("tiny", T=200, N=300)
+        x = (x * (1.0 + i)).contiguous()
+        xh, wh = x.pin_memory(), w.pin_memory()
+        yh = torch.empty((200, 300), dtype=torch.float32).pin_memory()
+        sq.sq_linear(xh, wh, wl.alpha, out_dtype=torch.float32, y=yh, workspace=ws)
+        outs.append((xh, wh, yh))
+        refs.append(oracle.linear(synth.host_array(x), synth.host_array(w), wl.alpha)["y"])
+    torch.cuda.synchronize()
+    for (_, _, yh), ref in zip(outs, refs):
+        assert_f32_close(yh.numpy(), ref, "back-to-back sq_linear")
+
+
 def _rows(T, n=6, seed=0):
     rng = np.random.default_rng(seed)
     return np.unique(np.concatenate([[0, T - 1], rng.choice(T, n, replace=False)]))

@@ -16,8 +16,8 @@ namespace sq {
 
 // ============================================================== per-tensor codes
 // Same layout as the column-maximum kernel: each lane owns VEC consecutive
-// columns (one 16-byte load per row), 8 warps stride over a chunk of rows with
-// 8 rows per warp in flight, about one wave of blocks. Every lane therefore
+// columns (one 16-byte load per row), 8 warps stride over a chunk of rows in
+// double-buffered batches of 4 rows per warp, about one wave of blocks. Every lane therefore
 // needs the multipliers of its own VEC columns only, kept in registers.
 //
 // Codes. One scale for the whole tensor, so the two multipliers fold into one:
@@ -80,16 +80,21 @@ per_tensor_quant_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t col
     const int64_t row_bytes = cols * (int64_t)sizeof(T);
     const uint8_t* p = x + col * (int64_t)sizeof(T);
 
-    for (int64_t r = r_begin + warp; r < r_end; r += 8 * kAbsmaxRowsInFlight) {
-        RawChunk<T> v[kAbsmaxRowsInFlight];
+    // Batches of kAbsmaxBatch rows per warp, double-buffered: the next batch's
+    // loads are issued before the current one is converted.
+    constexpr int B = kAbsmaxBatch;
+    constexpr int64_t step = 8 * B;
+    RawChunk<T> v[B], nxt[B];
+    int64_t r = r_begin + warp;
 #pragma unroll
-        for (int u = 0; u < kAbsmaxRowsInFlight; ++u) {
-            const int64_t rr = r + 8 * u;
-            // one 16-byte load: 8 bf16 or 4 fp32 values (the first half of an fp32 RawChunk)
-            if (rr < r_end) v[u].a = ld_stream_v4(p + rr * row_bytes);
-        }
+    for (int u = 0; u < B; ++u)
+        if (r + 8 * u < r_end) v[u].a = ld_stream_v4(p + (r + 8 * u) * row_bytes);   // 16 bytes: 8 bf16 or 4 fp32
+    for (; r < r_end; r += step) {
 #pragma unroll
-        for (int u = 0; u < kAbsmaxRowsInFlight; ++u) {
+        for (int u = 0; u < B; ++u)
+            if (r + step + 8 * u < r_end) nxt[u].a = ld_stream_v4(p + (r + step + 8 * u) * row_bytes);
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
             const int64_t rr = r + 8 * u;
             if (rr >= r_end) continue;
             uint32_t t[VEC];
@@ -125,8 +130,8 @@ per_tensor_quant_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t col
                         f2_unpack(c2[e / 2], c0, c1);
                         float qv = __fmul_rn(v[u].get(e), (e & 1) ? c1 : c0);
                         qv = fminf(fmaxf(qv, -127.0f), 127.0f);
-                        const float d = __fsub_rn(qv, __fsub_rn(__fadd_rn(qv, kMagic), kMagic));
-                        if (fabsf(d) >= 0.5f - kTieGuard) t[e] = exact_code_pt(v[u].get(e), s, col + e, scale);
+                        const float dd = __fsub_rn(qv, __fsub_rn(__fadd_rn(qv, kMagic), kMagic));
+                        if (fabsf(dd) >= 0.5f - kTieGuard) t[e] = exact_code_pt(v[u].get(e), s, col + e, scale);
                     }
                 }
             }
@@ -140,6 +145,8 @@ per_tensor_quant_kernel(const uint8_t* __restrict__ x, int64_t rows, int64_t col
                     __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
             }
         }
+#pragma unroll
+        for (int u = 0; u < B; ++u) v[u] = nxt[u];
     }
 }
 

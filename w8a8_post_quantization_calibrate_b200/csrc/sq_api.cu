@@ -4,7 +4,9 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include <cuda_runtime.h>
 
@@ -103,6 +105,40 @@ LinearLayout linear_layout(int64_t M, int64_t N, int64_t K, sq_dtype in_dt, sq_d
     return L;
 }
 
+// Host operands are staged by a copy stream of the library (one per device),
+// so that the next call's input copies overlap this call's GEMM and output
+// copy. Two events per workspace order the staging: inputs_ready (the copies
+// are done; the compute waits for it) and inputs_free (the last kernel that
+// reads the staged inputs is done; the next call's copies wait for it).
+struct CopyState {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t inputs_ready = nullptr;
+    cudaEvent_t inputs_free = nullptr;
+};
+std::mutex g_copy_mu;
+cudaStream_t g_copy_stream[64] = {};
+std::map<std::pair<int, const void*>, CopyState> g_copy_state;
+
+sq_status copy_state(const void* ws, CopyState& out) {
+    const int dev = device_info().device;
+    std::lock_guard<std::mutex> lk(g_copy_mu);
+    cudaError_t e;
+    if (!g_copy_stream[dev & 63]) {
+        if ((e = cudaStreamCreateWithFlags(&g_copy_stream[dev & 63], cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "create the copy stream");
+    }
+    CopyState& c = g_copy_state[{dev, ws}];
+    if (!c.inputs_ready) {
+        if ((e = cudaEventCreateWithFlags(&c.inputs_ready, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "create an event");
+        if ((e = cudaEventCreateWithFlags(&c.inputs_free, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "create an event");
+    }
+    c.stream = g_copy_stream[dev & 63];
+    out = c;
+    return SQ_OK;
+}
+
 // true if the pointer is usable by kernels (device or managed memory).
 bool is_device_ptr(const void* p) {
     cudaPointerAttributes a;
@@ -147,15 +183,24 @@ sq_status linear_impl(const void* x, const void* w, sq_dtype in_dt, int64_t M, i
     const void* wd = w;
     void* yd = y;
     cudaError_t e;
-    if (!is_device_ptr(x)) {
-        xd = base + L.x_stage;
-        if ((e = cudaMemcpyAsync(const_cast<void*>(xd), x, (size_t)M * K * ies, cudaMemcpyHostToDevice, st)) != cudaSuccess)
-            return cuda_fail(e, "copy x to device");
-    }
-    if (!is_device_ptr(w)) {
-        wd = base + L.w_stage;
-        if ((e = cudaMemcpyAsync(const_cast<void*>(wd), w, (size_t)N * K * ies, cudaMemcpyHostToDevice, st)) != cudaSuccess)
-            return cuda_fail(e, "copy w to device");
+    const bool x_host = !is_device_ptr(x), w_host = !is_device_ptr(w);
+    CopyState cs;
+    if (x_host || w_host) {
+        sq_status r0 = copy_state(ws, cs);
+        if (r0 != SQ_OK) return r0;
+        if ((e = cudaStreamWaitEvent(cs.stream, cs.inputs_free, 0)) != cudaSuccess) return cuda_fail(e, "wait for the staging");
+        if (x_host) {
+            xd = base + L.x_stage;
+            if ((e = cudaMemcpyAsync(const_cast<void*>(xd), x, (size_t)M * K * ies, cudaMemcpyHostToDevice, cs.stream)) != cudaSuccess)
+                return cuda_fail(e, "copy x to device");
+        }
+        if (w_host) {
+            wd = base + L.w_stage;
+            if ((e = cudaMemcpyAsync(const_cast<void*>(wd), w, (size_t)N * K * ies, cudaMemcpyHostToDevice, cs.stream)) != cudaSuccess)
+                return cuda_fail(e, "copy w to device");
+        }
+        if ((e = cudaEventRecord(cs.inputs_ready, cs.stream)) != cudaSuccess) return cuda_fail(e, "record the copies");
+        if ((e = cudaStreamWaitEvent(st, cs.inputs_ready, 0)) != cudaSuccess) return cuda_fail(e, "wait for the copies");
     }
     const bool y_host = !is_device_ptr(y);
     if (y_host) yd = base + L.y_stage;
@@ -175,6 +220,8 @@ sq_status linear_impl(const void* x, const void* w, sq_dtype in_dt, int64_t M, i
     if ((r = smooth_factors_impl(xmax, wmax, K, alpha, eps, s, st)) != SQ_OK) return r;
     if ((r = fold_quant_weights_impl(wd, in_dt, N, K, s, wq, wsc, st)) != SQ_OK) return r;
     if ((r = smooth_quant_act_impl(xd, in_dt, M, K, s, xq, xs, st)) != SQ_OK) return r;
+    if ((x_host || w_host) && (e = cudaEventRecord(cs.inputs_free, st)) != cudaSuccess)
+        return cuda_fail(e, "record the end of the staged inputs' use");
     if ((r = gemm_dispatch(xq, xs, wq, wsc, M, N, K, yd, out_dt, base + L.gemm_ws, L.gemm_ws_bytes, st)) != SQ_OK)
         return r;
     if (y_host) {
