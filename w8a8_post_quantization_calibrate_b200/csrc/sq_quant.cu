@@ -470,7 +470,9 @@ __device__ __forceinline__ float group_max(float v, float* red, int grp, int wig
 template <int R>
 constexpr int row_fast_threads() { return 32 * R > 256 ? 32 * R : 256; }
 
-template <typename T, int MODE, int R, int CPL>
+// PF: double-buffer the row in registers (the next row's loads are issued
+// before the current row is processed).
+template <typename T, int MODE, int R, int CPL, bool PF>
 __global__ void __launch_bounds__(row_fast_threads<R>(), R >= 16 ? 1 : (R >= 8 ? 2 : 4))
 row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
                       int8_t* __restrict__ q, float* __restrict__ scale_out, float eps,
@@ -505,9 +507,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
 
     const uint64_t mag2 = f2_pack(kMagic, kMagic);
     int bank = 0, bank64 = 0;
-    // Long rows (R >= 8) double-buffer the row in registers: the next row's
-    // loads are issued before the current row is processed.
-    constexpr bool kPrefetch = R >= 8;
+    constexpr bool kPrefetch = PF;
     const int64_t stride = (int64_t)gridDim.x * groups;
     RawChunk<T> nxt[CPL];
     if (kPrefetch) {
@@ -729,16 +729,15 @@ sq_status launch_row_quant_exact(const void* in, int64_t rows, int64_t K, const 
     }
 }
 
-template <typename T, int MODE, int R>
+template <typename T, int MODE, int R, int CPL = RowFastCPL<T>::value, bool PF = (R >= 8)>
 sq_status launch_row_quant_fast_inst(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
                                      float* scale, cudaStream_t st, float eps, float* r_out) {
-    constexpr int CPL = RowFastCPL<T>::value;
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const int threads = 32 * R > 256 ? 32 * R : 256;
     const int groups = threads / (32 * R);
     const size_t smem = (size_t)K * 6 + (size_t)groups * 2 * R * (sizeof(float) + (MODE == kNorm ? sizeof(double) : 0));
-    auto kern = row_quant_fast_kernel<T, MODE, R, CPL>;
+    auto kern = row_quant_fast_kernel<T, MODE, R, CPL, PF>;
     if (!attr_done[di.device & 63]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)(kFastMaxK * 6 + 1024));
