@@ -197,6 +197,7 @@ GEMM_SHAPES = [
     (1, 16, 16), (1, 128, 128), (3, 200, 272), (8, 1000, 512), (16, 1024, 4096), (16, 300, 1040),
     (17, 256, 128), (100, 300, 272), (128, 256, 128), (129, 257, 144), (256, 512, 1024),
     (300, 1000, 2048), (1024, 768, 4096), (129, 4096, 1024), (513, 1000, 1040),
+    (1024, 9728, 512), (777, 10000, 272), (2048, 12288, 1024),
 ]
 
 
