@@ -467,6 +467,87 @@ __device__ __forceinline__ float group_max(float v, float* red, int grp, int wig
     return v;
 }
 
+// The rarely taken paths of the row kernel. Kernels that keep one row in
+// registers call them out of line (the hot loop stays small in the
+// instruction cache); kernels that also hold the next row (PF) inline them, as
+// a call would make the live prefetch registers spill. A chunk is passed by value.
+
+// max_e |v_e| of one chunk, every value exact.
+template <typename T, int MODE>
+__device__ __forceinline__ float exact_chunk_max_in(const RawChunk<T>& ch, const float* __restrict__ s8, float rn) {
+    float ex = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(ch.get(e), __ldg(s8 + e), rn));
+    return ex;
+}
+template <typename T, int MODE>
+__device__ __noinline__ float exact_chunk_max_out(const RawChunk<T> ch, const float* __restrict__ s8, float rn) {
+    return exact_chunk_max_in<T, MODE>(ch, s8, rn);
+}
+
+// Exact codes of one chunk, packed 8 per uint2 (zero codes for a zero scale).
+template <typename T, int MODE>
+__device__ __forceinline__ uint2 exact_chunk_codes_in(const RawChunk<T>& ch, const float* __restrict__ s8, float scale,
+                                                      float rn, bool zero) {
+    uint32_t b[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) b[e] = zero ? 0u : exact_code<MODE>(ch.get(e), __ldg(s8 + e), scale, rn);
+    return make_uint2(b[0] | b[1] << 8 | b[2] << 16 | b[3] << 24, b[4] | b[5] << 8 | b[6] << 16 | b[7] << 24);
+}
+template <typename T, int MODE>
+__device__ __noinline__ uint2 exact_chunk_codes_out(const RawChunk<T> ch, const float* __restrict__ s8, float scale,
+                                                    float rn, bool zero) {
+    return exact_chunk_codes_in<T, MODE>(ch, s8, scale, rn, zero);
+}
+
+// Near-tie repair of one chunk's packed codes: every element whose fast
+// quotient lies within the guard of a half-integer gets its exact code.
+template <typename T, int MODE>
+__device__ __forceinline__ uint2 fix_near_ties_in(const RawChunk<T>& ch, uint2 codes, const float* __restrict__ m_lo,
+                                                  const float* __restrict__ m_hi, const float* __restrict__ s8, float r,
+                                                  float rn, float scale) {
+    const float4 a = *reinterpret_cast<const float4*>(m_lo);
+    const float4 b = *reinterpret_cast<const float4*>(m_hi);
+    const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float xe = MODE == kNorm ? __fmul_rn(ch.get(e), rn) : ch.get(e);
+        const float qv = __fmul_rn(__fmul_rn(xe, mv[e]), r);
+        const float d = __fsub_rn(qv, __fsub_rn(__fadd_rn(qv, kMagic), kMagic));
+        if (fabsf(d) >= 0.5f - kTieGuard) {
+            const uint32_t code = exact_code<MODE>(ch.get(e), __ldg(s8 + e), scale, rn);
+            const int sh = 8 * (e & 3);
+            uint32_t& w = (e < 4) ? codes.x : codes.y;
+            w = (w & ~(0xffu << sh)) | (code << sh);
+        }
+    }
+    return codes;
+}
+template <typename T, int MODE>
+__device__ __noinline__ uint2 fix_near_ties_out(const RawChunk<T> ch, uint2 codes, const float* __restrict__ m_lo,
+                                                const float* __restrict__ m_hi, const float* __restrict__ s8, float r,
+                                                float rn, float scale) {
+    return fix_near_ties_in<T, MODE>(ch, codes, m_lo, m_hi, s8, r, rn, scale);
+}
+
+template <typename T, int MODE, bool OUT>
+__device__ __forceinline__ float exact_chunk_max(const RawChunk<T>& ch, const float* s8, float rn) {
+    if constexpr (OUT) return exact_chunk_max_out<T, MODE>(ch, s8, rn);
+    else return exact_chunk_max_in<T, MODE>(ch, s8, rn);
+}
+template <typename T, int MODE, bool OUT>
+__device__ __forceinline__ uint2 exact_chunk_codes(const RawChunk<T>& ch, const float* s8, float scale, float rn,
+                                                   bool zero) {
+    if constexpr (OUT) return exact_chunk_codes_out<T, MODE>(ch, s8, scale, rn, zero);
+    else return exact_chunk_codes_in<T, MODE>(ch, s8, scale, rn, zero);
+}
+template <typename T, int MODE, bool OUT>
+__device__ __forceinline__ uint2 fix_near_ties(const RawChunk<T>& ch, uint2 codes, const float* m_lo, const float* m_hi,
+                                               const float* s8, float r, float rn, float scale) {
+    if constexpr (OUT) return fix_near_ties_out<T, MODE>(ch, codes, m_lo, m_hi, s8, r, rn, scale);
+    else return fix_near_ties_in<T, MODE>(ch, codes, m_lo, m_hi, s8, r, rn, scale);
+}
+
 template <int R>
 constexpr int row_fast_threads() { return 32 * R > 256 ? 32 * R : 256; }
 
@@ -592,9 +673,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
 #pragma unroll
             for (int i = 0; i < CPL; ++i) {
                 const int64_t c = gl + (int64_t)i * 32 * R;
-                if (c < nchunks)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), rn));
+                if (c < nchunks) ex = fmaxf(ex, exact_chunk_max<T, MODE, !PF>(raw[i], s + c * 8, rn));
             }
             const float a = group_max<R>(ex, red, grp, wig, lane, bank);
             bank ^= 1;
@@ -602,14 +681,9 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
 #pragma unroll
             for (int i = 0; i < CPL; ++i) {
                 const int64_t c = gl + (int64_t)i * 32 * R;
-                if (c < nchunks) {
-                    uint32_t b[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        b[e] = a == 0.0f ? 0u : exact_code<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), scale, rn);
-                    *reinterpret_cast<uint2*>(rq + c * 8) =
-                        make_uint2(b[0] | b[1] << 8 | b[2] << 16 | b[3] << 24, b[4] | b[5] << 8 | b[6] << 16 | b[7] << 24);
-                }
+                if (c < nchunks)
+                    *reinterpret_cast<uint2*>(rq + c * 8) = exact_chunk_codes<T, MODE, !PF>(raw[i], s + c * 8, scale, rn,
+                                                                                     a == 0.0f);
             }
             if (gl == 0) scale_out[row] = scale;
             continue;
@@ -622,8 +696,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
         for (int i = 0; i < CPL; ++i) {
             if (cm[i] >= tau) {
                 const int64_t c = gl + (int64_t)i * 32 * R;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ex = fmaxf(ex, exact_abs<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), rn));
+                ex = fmaxf(ex, exact_chunk_max<T, MODE, !PF>(raw[i], s + c * 8, rn));
             }
         }
         const float amax = group_max<R>(ex, red, grp, wig, lane, bank);
@@ -657,19 +730,12 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
                     near_tie |= fabsf(d0) >= 0.5f - kTieGuard;
                     near_tie |= fabsf(d1) >= 0.5f - kTieGuard;
                 }
-                if (near_tie) {
-                    const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float xe = MODE == kNorm ? __fmul_rn(raw[i].get(e), rn) : raw[i].get(e);
-                        const float qv = __fmul_rn(__fmul_rn(xe, mv[e]), r);
-                        const float d = __fsub_rn(qv, __fsub_rn(__fadd_rn(qv, kMagic), kMagic));
-                        if (fabsf(d) >= 0.5f - kTieGuard) t[e] = exact_code<MODE>(raw[i].get(e), __ldg(s + c * 8 + e), scale, rn);
-                    }
-                }
-                const uint32_t lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-                const uint32_t hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
-                *reinterpret_cast<uint2*>(rq + c * 8) = make_uint2(lo, hi);
+                uint2 codes;
+                codes.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+                codes.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+                if (near_tie)
+                    codes = fix_near_ties<T, MODE, !PF>(raw[i], codes, mul_lo + c * 4, mul_hi + c * 4, s + c * 8, r, rn, scale);
+                *reinterpret_cast<uint2*>(rq + c * 8) = codes;
             }
         }
         if (gl == 0) scale_out[row] = scale;
