@@ -1,0 +1,186 @@
+"""The streamed row kernel (bf16 rows of 2064 to 16384 channels, staged in
+shared memory by bulk copies): fold + quantize (a3), smooth + quantize (a4) and
+RMSNorm + quantize against the CPU oracle, through the C ABI.
+
+Bar: codes and scales bit-exact. The shapes cover every group width the kernel
+uses (2, 4 and 8 warps per row) and every chunk count per lane (5 to 8), rows
+padded to whole lanes and rows that fill them exactly, and many rows per
+group (the ring of row slots wraps many times); the
+special rows drive its exact paths: near-ties of the fast quotient, many
+candidates for the row maximum, tiny, denormal, zero and huge rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import assert_bitexact_f32, assert_equal, bits32, host
+from w8a8_post_quantization_calibrate_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from w8a8_post_quantization_calibrate_b200 import sq  # noqa: E402
+
+DEV = torch.device("cuda", 0)
+BF16 = torch.bfloat16
+
+# (rows, K) -> warps per row, chunks per lane (padded chunks): 2064 -> 2, 5 (62);
+# 4096 -> 2, 8; 4112 -> 4, 5 (126); 6144 -> 4, 6; 6160 -> 4, 7 (126); 8192 -> 4, 8;
+# 11008 -> 8, 6 (160); 12304 -> 8, 7 (254); 16384 -> 8, 8.
+SHAPES = [(1, 2064), (37, 4096), (2500, 4096), (300, 4112), (17, 6144), (9, 6160), (200, 8192), (33, 11008),
+          (5, 12304), (3, 16384), (70, 16384)]
+
+
+def dev(t):
+    return t.contiguous().to(DEV)
+
+
+def s_for(K, seed):
+    return np.random.default_rng(seed).uniform(0.05, 20.0, K).astype(np.float32)
+
+
+def outlier_x(T, K, seed, n_out=3, scale=50.0):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(T, K, generator=g)
+    x[:, torch.randperm(K, generator=g)[:n_out]] *= scale
+    return x.to(BF16)
+
+
+def check_fold(w, s, what):
+    q, sc = sq.sq_fold_quant_weights(dev(w), dev(torch.from_numpy(s)))
+    oq, osc = oracle.fold_quant_weights(synth.host_array(w), s)
+    assert_equal(host(q), oq, f"{what} codes")
+    assert_bitexact_f32(host(sc), osc, f"{what} scales")
+
+
+def check_smooth(x, s, what):
+    q, sc = sq.sq_smooth_quant_act(dev(x), dev(torch.from_numpy(s)))
+    oq, osc = oracle.smooth_quant_act(synth.host_array(x), s)
+    assert_equal(host(q), oq, f"{what} codes")
+    assert_bitexact_f32(host(sc), osc, f"{what} scales")
+
+
+def check_norm(x, gf, eps, what):
+    xq, xs, r = sq.sq_rmsnorm_quant_act(dev(x), dev(torch.from_numpy(gf)), eps)
+    hx = synth.host_array(x)
+    _, _, o_r = oracle.rmsnorm_quant_act(hx, gf, eps)
+    g_r = host(r)
+    ulps = np.abs(bits32(g_r).astype(np.int64) - bits32(o_r).astype(np.int64))
+    assert ulps.max(initial=0) <= 1, f"{what}: inv_rms {ulps.max()} ulps apart"
+    oq, osc, _ = oracle.rmsnorm_quant_act(hx, gf, eps, r_in=g_r)
+    assert_equal(host(xq), oq, f"{what} codes")
+    assert_bitexact_f32(host(xs), osc, f"{what} scales")
+
+
+@pytest.mark.parametrize("rows,K", SHAPES)
+def test_fold_stream(rows, K):
+    g = torch.Generator().manual_seed(rows + 3 * K)
+    w = (torch.randn(rows, K, generator=g) * 0.05).to(BF16)
+    if rows > 2:
+        w[0] = 0
+        w[2, K // 3:] = 0
+    check_fold(w, s_for(K, K + 1), f"fold {rows}x{K}")
+
+
+@pytest.mark.parametrize("rows,K", SHAPES)
+def test_smooth_stream(rows, K):
+    x = outlier_x(rows, K, seed=K + rows)
+    if rows > 2:
+        x[1] = 0
+        x[2, : K // 2] = 0
+    check_smooth(x, s_for(K, K), f"smooth {rows}x{K}")
+
+
+@pytest.mark.parametrize("rows,K", SHAPES)
+def test_norm_stream(rows, K):
+    x = outlier_x(rows, K, seed=rows * 5 + K, scale=30.0)
+    if rows > 2:
+        x[1] = 0
+    gain = np.random.default_rng(K).uniform(0.5, 1.5, K).astype(np.float32)
+    check_norm(x, oracle.fold_norm_gain(gain, s_for(K, K + 7)), 1e-6, f"norm {rows}x{K}")
+
+
+def _tie_targets(scale):
+    """fp32 values a few ulps either side of (k + 1/2) * scale, k = 0..126."""
+    out = []
+    for k in range(127):
+        v0 = np.float32((k + 0.5) * float(scale))
+        for d in range(-3, 4):
+            out.append(np.float32(v0 + d * np.spacing(v0)))
+    return np.array(out, np.float32)
+
+
+@pytest.mark.parametrize("K", [4096, 8192, 16384])
+def test_near_ties(K):
+    """With x = 1 the folded value is s itself and the smoothed value RN(1/s):
+    choosing s puts hundreds of quotients within a few ulps of k + 1/2, in
+    every lane position of the row."""
+    scale = np.float32(30.0) / np.float32(127.0)
+    t = _tie_targets(scale)
+    rng = np.random.default_rng(K)
+    pos = rng.permutation(np.arange(1, K))[: len(t)]
+    s_fold = rng.uniform(0.01, 0.2, K).astype(np.float32)
+    s_fold[0] = 30.0
+    s_fold[pos] = t
+    w = torch.ones(3, K, dtype=BF16)
+    w[1] = -1.0
+    w[2, ::2] = 0.5
+    check_fold(w, s_fold, f"fold near ties K={K}")
+    s_smooth = (np.float32(1.0) / s_fold).astype(np.float32)
+    check_smooth(torch.ones(2, K, dtype=BF16), s_smooth, f"smooth near ties K={K}")
+
+
+@pytest.mark.parametrize("K", [4096, 6160, 16384])
+def test_many_candidates_for_the_maximum(K):
+    """Smoothed rows whose largest values differ by a few ulps, spread over
+    all lanes and warps of the group: only exact divisions can tell them
+    apart, so the scale is right only if every candidate is resolved."""
+    rng = np.random.default_rng(K + 1)
+    base = np.float32(3.0)
+    s = np.full(K, base, np.float32)
+    n = 300
+    pos = rng.choice(K, n, replace=False)
+    s[pos] = base + (rng.integers(-4, 5, n) * np.spacing(base)).astype(np.float32)
+    x = torch.ones(4, K, dtype=BF16)
+    x[1] = -1.0
+    x[2] = float(np.float32(1.5))
+    x[3, ::3] = 7.0
+    check_smooth(x, s, f"candidates K={K}")
+    check_fold(x, s, f"fold near-equal maxima K={K}")
+
+
+def test_tiny_denormal_zero_and_huge_rows():
+    K = 4096
+    g = torch.Generator().manual_seed(12)
+    x = torch.randn(9, K, generator=g)
+    x[0] *= 1e-33
+    x[1] *= 1e-38
+    x[2] = 0.0
+    x[2, 5] = 1e-39
+    x[3, 7] = 1e30
+    x[4] *= 1e-20
+    x[5, :16] = 0.0
+    x[6] *= 1e30
+    x[7] = 0.0
+    x = x.to(BF16)
+    s = s_for(K, 77)
+    check_smooth(x, s, "extreme rows, smooth")
+    check_fold(x, s, "extreme rows, fold")
+    gf = oracle.fold_norm_gain(np.ones(K, np.float32), s_for(K, 1))
+    for eps in (1e-6, 1.0):
+        check_norm(x, gf, eps, f"extreme rows, norm eps={eps}")
+
+
+def test_keep_mask_fold_is_the_bulk_quantizer():
+    """The decomposition's bulk quantizer (a 0/1 multiplier) on the streamed path."""
+    K = 4096
+    x = outlier_x(64, K, seed=5, n_out=6, scale=20.0)
+    keep = np.ones(K, np.float32)
+    keep[np.random.default_rng(5).choice(K, 6, replace=False)] = 0.0
+    q, sc = sq.sq_quant_bulk(dev(x), dev(torch.from_numpy(keep)))
+    oq, osc = oracle.quant_bulk(synth.host_array(x), keep)
+    assert_equal(host(q), oq, "bulk codes")
+    assert_bitexact_f32(host(sc), osc, "bulk scales")

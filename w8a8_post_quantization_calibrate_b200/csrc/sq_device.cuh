@@ -87,6 +87,34 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
     }
 }
 
+// The same bounded wait for threads with nothing else to do: each try_wait
+// may suspend the thread (up to 0.2 ms) until the phase completes, instead of
+// returning at once, so that waiting warps do not take issue slots from the
+// warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity), "r"(200000u) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, long long limit,
+                                                volatile int* abort, unsigned int site) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit) {
+            *abort = 1;
+            record_status(SQ_ERR_TIMEOUT, site);
+            return false;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // The library's kernels are launched with programmatic stream serialization:
 // a kernel may be scheduled while the previous kernel in the stream is still

@@ -742,6 +742,341 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
     }
 }
 
+// ============================================================== the streamed row kernel (bf16)
+// bf16 rows of 2064 to 16384 elements. One CTA of 16 warps per SM, in groups
+// of R warps; a group quantizes one row at a time, lane l of the group owning
+// the 8-element chunks l, l + 32R, ... (CPL of them: the row is padded with
+// zeros to 32 R CPL chunks, so the unrolled loops need no bounds checks and
+// only the stores are predicated). Rows reach shared memory through a ring of
+// ns slots per group (two in practice), each filled by one bulk copy
+// (cp.async.bulk, its bytes counted on the slot's mbarrier) that the group's
+// first lane issues ns - 1 rows ahead. DRAM latency is hidden without a second
+// row in registers, and the registers hold the row's values instead:
+//   fold   v_j = RN(x_j * s_j)                  exact
+//   norm   v_j = RN(RN(x_j * r_t) * g'_j)       exact
+//   smooth v'_j = RN(x_j * RN(1/s_j))           within 3 * 2^-24 |v_j| of v_j = RN(x_j / s_j)
+// formed once (pass 1) as fp32 pairs. The row maximum is therefore exact for
+// fold and norm. For smooth, the elements with |v'_j| >= m'(1 - 2^-20) (m' the
+// maximum of the |v'|) get their exact value from an IEEE division; the true
+// maximum is always among them, since m' <= a(1 + 3 * 2^-24) and the element
+// attaining a has |v'| >= a(1 - 3 * 2^-24).
+//
+// Codes (pass 2): with r = RN(1/scale), t = RN(v * r + 1.5 * 2^23) holds
+// k = round-half-even(v * r) in its low mantissa bits, and d = RN(v * r - k)
+// is the distance to it. v * r (one rounding, inside the fused multiply-add)
+// is within 1.2e-5 of q* = RN(v / scale) for exact v and within 3.5e-5 for
+// smooth's v', so k is the code of q* unless |d| >= 0.5 - 2^-13. Such elements
+// (about one per 4096) get the IEEE-division code after their chunk's store,
+// recomputed from the copy of the row still in shared memory; chunks needing
+// exact work are collected in a bit mask, so the rare paths stay out of the
+// unrolled loops. Rows whose maximum is below 2^-90 (all-zero rows included)
+// are quantized entirely with exact divisions, as in the register kernel.
+constexpr int kRingThreads = 512;
+constexpr int kRingCPL = 8;
+constexpr size_t kRingSmemMax = 231424;   // dynamic shared memory of one CTA (226 KB of the 227 KB opt-in)
+constexpr float kRingCandidate = 1.0f - 1.0f / 1048576.0f;
+
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ float bf16_elem(const uint4& w, int e) {
+    const uint32_t u = e < 2 ? w.x : e < 4 ? w.y : e < 6 ? w.z : w.w;
+    return (e & 1) ? bf16_hi(u) : bf16_lo(u);
+}
+
+// Elements (2p, 2p+1) of a 16-byte bf16 chunk as an fp32 pair.
+__device__ __forceinline__ uint64_t bf16_pair(const uint4& w, int p) {
+    const uint32_t u = p == 0 ? w.x : p == 1 ? w.y : p == 2 ? w.z : w.w;
+    return f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+// The R warps of a group agree on `ok`: a named barrier with an AND reduction.
+template <int R>
+__device__ __forceinline__ bool group_all(bool ok, int grp) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+                 "bar.red.and.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)ok), "r"(1 + grp), "r"(32 * R) : "memory");
+    return r != 0;
+}
+
+template <int MODE, int R, int CPL>
+__global__ void __launch_bounds__(kRingThreads, 1)
+row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
+                      int8_t* __restrict__ q, float* __restrict__ scale_out, float eps, float* __restrict__ r_out,
+                      int ns, long long wait_limit) {
+    constexpr int G = kRingThreads / (32 * R);   // groups per CTA
+    constexpr int NCP = 32 * R * CPL;            // chunks of a row padded to whole lanes
+    constexpr uint32_t SLOT = NCP * 16u;         // bytes of one ring slot
+    extern __shared__ __align__(128) uint8_t ring_smem[];
+    const int64_t nchunks = K >> 3;
+    const int nch = (int)nchunks;
+    const uint32_t row_bytes = (uint32_t)K * 2u;
+    float* mul_lo = reinterpret_cast<float*>(ring_smem);         // [NCP][4]: m_j of elements 0..3
+    float* mul_hi = mul_lo + NCP * 4;                            // [NCP][4]: elements 4..7
+    uint8_t* slots = ring_smem + NCP * 32;                       // [G][ns][SLOT]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(slots + (size_t)G * ns * SLOT);   // [G][ns]
+    float* red = reinterpret_cast<float*>(bars + G * ns);        // [G][2][R]
+    double* red64 = reinterpret_cast<double*>(red + G * 2 * R);  // [G][2][R]
+    __shared__ int abort_sh, never_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = warp / R, wig = warp % R;
+    const int gl = wig * 32 + lane;
+    uint8_t* my_slots = slots + (size_t)grp * ns * SLOT;
+    const uint32_t bar0 = smem_u32(bars + grp * ns);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < G * ns; ++i) mbar_init(smem_u32(bars + i), 1);
+        abort_sh = 0;
+        never_sh = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+
+    const int64_t stride = (int64_t)gridDim.x * G;
+    const int64_t row0 = (int64_t)blockIdx.x * G + grp;
+    if (gl == 0) {
+        for (int j = 0; j < ns; ++j) {
+            const int64_t row = row0 + (int64_t)j * stride;
+            if (row < rows) {
+                mbar_arrive_expect_tx(bar0 + 8u * j, row_bytes);
+                bulk_copy_g2s(smem_u32(my_slots + (size_t)j * SLOT), in + row * K, row_bytes, bar0 + 8u * j);
+            }
+        }
+    }
+    // multipliers, zero past the row's end; the slots' padding (never
+    // written by a copy) is zeroed once, so every lane handles CPL chunks
+    // without bounds checks and the padding adds nothing to any maximum
+    for (int c = threadIdx.x; c < NCP; c += kRingThreads) {
+        float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f), b = a;
+        if (c < nch) {
+            a = __ldg(reinterpret_cast<const float4*>(s + c * 8));
+            b = __ldg(reinterpret_cast<const float4*>(s + c * 8 + 4));
+        }
+        if (MODE == kSmooth && c < nch) {
+            a = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
+            b = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
+        }
+        *reinterpret_cast<float4*>(mul_lo + c * 4) = a;
+        *reinterpret_cast<float4*>(mul_hi + c * 4) = b;
+    }
+    {
+        const int tail = (int)((SLOT - row_bytes) / 16u);
+        for (int i = threadIdx.x; i < G * ns * tail; i += kRingThreads)
+            *reinterpret_cast<uint4*>(slots + (size_t)(i / tail) * SLOT + row_bytes + (size_t)(i % tail) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+
+    const uint64_t mag2 = f2_pack(kMagic, kMagic);
+    int bank = 0, bank64 = 0;
+    int it = 0, sl = 0, ps = ns - 1;   // iteration, its slot, the previous iteration's slot
+    uint32_t parity = 0;
+    bool failed = false;
+    for (int64_t row = row0; row < rows; row += stride, ++it) {
+        const bool ok = mbar_wait_sleep(bar0 + 8u * sl, parity, wait_limit, &abort_sh, SITE_QUANT_WAIT);
+        __syncwarp();   // the barrier below is warp-aligned
+        if (!group_all<R>(ok, grp)) {
+            failed = true;
+            break;
+        }
+        // every warp of the group is done with the previous row's slot: refill it
+        if (it > 0 && gl == 0) {
+            const int64_t nr = row + (int64_t)(ns - 1) * stride;
+            if (nr < rows) {
+                mbar_arrive_expect_tx(bar0 + 8u * ps, row_bytes);
+                bulk_copy_g2s(smem_u32(my_slots + (size_t)ps * SLOT), in + nr * K, row_bytes, bar0 + 8u * ps);
+            }
+        }
+        const uint8_t* src = my_slots + (size_t)sl * SLOT;
+        ps = sl;
+        if (++sl == ns) {
+            sl = 0;
+            parity ^= 1u;
+        }
+
+        // ---- RMSNorm factor of the row (sum of squares in fp64, every square exact)
+        float rn = 1.0f;
+        if (MODE == kNorm) {
+            double ss = 0.0;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int c = gl + i * 32 * R;
+                const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const double v = (double)bf16_elem(w, e);
+                    ss = __fma_rn(v, v, ss);
+                }
+            }
+            ss = group_sum<R>(ss, red64, grp, wig, lane, bank64);
+            bank64 ^= 1;
+            rn = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)K), (double)eps))));
+            if (r_out != nullptr && gl == 0) r_out[row] = rn;
+        }
+        const uint64_t rn2 = f2_pack(rn, rn);
+
+        // ---- pass 1: the values, kept in registers, and their maximum
+        uint64_t v2[CPL][4];
+        float cm[CPL];
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = gl + i * 32 * R;
+            const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
+            const float4 a = *reinterpret_cast<const float4*>(mul_lo + c * 4);
+            const float4 b = *reinterpret_cast<const float4*>(mul_hi + c * 4);
+            const uint64_t mp[4] = {f2_pack(a.x, a.y), f2_pack(a.z, a.w), f2_pack(b.x, b.y), f2_pack(b.z, b.w)};
+            float cmax = 0.0f;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                uint64_t x2 = bf16_pair(w, p);
+                if (MODE == kNorm) x2 = f2_mul(x2, rn2);
+                v2[i][p] = f2_mul(x2, mp[p]);
+                float lo, hi;
+                f2_unpack(v2[i][p], lo, hi);
+                cmax = fmax3(cmax, fabsf(lo), fabsf(hi));
+            }
+            cm[i] = cmax;
+            m = fmaxf(m, cmax);
+        }
+        float amax = group_max<R>(m, red, grp, wig, lane, bank);
+        bank ^= 1;
+        int8_t* rq = q + row * K;
+
+        if (!(amax >= kSmallRow)) {
+            // zero, tiny or near-underflow row: exact maximum and codes
+            float ex = 0.0f;
+#pragma unroll 1
+            for (int i = 0; i < CPL; ++i) {
+                const int c = gl + i * 32 * R;
+                if (c < nch) {
+                    RawChunk<__nv_bfloat16> ch;
+                    ch.a = *reinterpret_cast<const uint4*>(src + c * 16);
+                    ex = fmaxf(ex, exact_chunk_max_in<__nv_bfloat16, MODE>(ch, s + c * 8, rn));
+                }
+            }
+            const float a = group_max<R>(ex, red, grp, wig, lane, bank);
+            bank ^= 1;
+            const float scale = a == 0.0f ? 1.0f : __fdiv_rn(a, 127.0f);
+#pragma unroll 1
+            for (int i = 0; i < CPL; ++i) {
+                const int c = gl + i * 32 * R;
+                if (c < nch) {
+                    RawChunk<__nv_bfloat16> ch;
+                    ch.a = *reinterpret_cast<const uint4*>(src + c * 16);
+                    *reinterpret_cast<uint2*>(rq + c * 8) =
+                        exact_chunk_codes_in<__nv_bfloat16, MODE>(ch, s + c * 8, scale, rn, a == 0.0f);
+                }
+            }
+            if (gl == 0) scale_out[row] = scale;
+            continue;
+        }
+
+        if (MODE == kSmooth) {
+            // exact values of the candidates (normally the maximum alone)
+            const float thr = __fmul_rn(amax, kRingCandidate);
+            uint32_t cand = 0;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) cand |= (cm[i] >= thr ? 1u : 0u) << i;
+            float ex = 0.0f;
+            while (cand) {
+                const int i = __ffs(cand) - 1;
+                cand &= cand - 1;
+                const int c = gl + i * 32 * R;
+                const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
+                const float4 a = *reinterpret_cast<const float4*>(mul_lo + c * 4);
+                const float4 b = *reinterpret_cast<const float4*>(mul_hi + c * 4);
+                const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x = bf16_elem(w, e);
+                    if (fabsf(__fmul_rn(x, mv[e])) >= thr) ex = fmaxf(ex, exact_abs<MODE>(x, __ldg(s + c * 8 + e), rn));
+                }
+            }
+            amax = group_max<R>(ex, red, grp, wig, lane, bank);
+            bank ^= 1;
+        }
+
+        // ---- pass 2: codes
+        const float scale = __fdiv_rn(amax, 127.0f);
+        const float r = __frcp_rn(scale);
+        const uint64_t r2 = f2_pack(r, r);
+        uint32_t ntm = 0;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = gl + i * 32 * R;
+            {
+                uint32_t t[8];
+                float dm = 0.0f;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const uint64_t t2 = f2_fma(v2[i][p], r2, mag2);
+                    const uint64_t d2 = f2_fma(v2[i][p], r2, f2_sub(mag2, t2));
+                    float t0, t1, d0, d1;
+                    f2_unpack(t2, t0, t1);
+                    f2_unpack(d2, d0, d1);
+                    t[2 * p] = __float_as_uint(t0);
+                    t[2 * p + 1] = __float_as_uint(t1);
+                    dm = fmax3(dm, fabsf(d0), fabsf(d1));
+                }
+                uint2 codes;
+                codes.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+                codes.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+                if (c < nch) *reinterpret_cast<uint2*>(rq + c * 8) = codes;
+                ntm |= (dm >= 0.5f - kTieGuard ? 1u : 0u) << i;   // (padding: d = 0)
+            }
+        }
+        if (gl == 0) scale_out[row] = scale;
+        // near ties: the same fast quotient recomputed per element; those
+        // within the guard get the IEEE-division code (same thread, later store)
+        while (ntm) {
+            const int i = __ffs(ntm) - 1;
+            ntm &= ntm - 1;
+            const int c = gl + i * 32 * R;
+            const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
+            const float4 a = *reinterpret_cast<const float4*>(mul_lo + c * 4);
+            const float4 b = *reinterpret_cast<const float4*>(mul_hi + c * 4);
+            const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float x = bf16_elem(w, e);
+                const float vf = MODE == kNorm ? __fmul_rn(__fmul_rn(x, rn), mv[e]) : __fmul_rn(x, mv[e]);
+                const float tf = __fmaf_rn(vf, r, kMagic);
+                const float df = __fmaf_rn(vf, r, __fsub_rn(kMagic, tf));
+                if (fabsf(df) >= 0.5f - kTieGuard)
+                    rq[c * 8 + e] = (int8_t)exact_code<MODE>(x, __ldg(s + c * 8 + e), scale, rn);
+            }
+        }
+    }
+
+    if (failed && gl == 0) {
+        // copies issued for rows this group will not consume: let them land
+        // before the CTA exits (bounded)
+        for (int j = it; j < it + ns - 1; ++j) {
+            const int64_t row = row0 + (int64_t)j * stride;
+            if (row < rows) mbar_wait(bar0 + 8u * (j % ns), (uint32_t)(j / ns) & 1u, wait_limit, &never_sh, SITE_QUANT_DRAIN);
+        }
+    }
+}
+
 // ============================================================== host side
 namespace {
 
@@ -821,11 +1156,77 @@ sq_status launch_row_quant_fast_inst(const void* in, int64_t rows, int64_t K, co
                       static_cast<const T*>(in), rows, K, s, q, scale, eps, r_out);
 }
 
+// The streamed kernel's shared memory: multipliers and ns row slots per group,
+// both padded to 32 * R * CPL chunks, the slots' mbarriers and the group
+// reduction slots.
+size_t ring_smem_bytes(int R, int CPL, int ns) {
+    const size_t G = (size_t)(kRingThreads / (32 * R));
+    const size_t ncp = (size_t)32 * R * CPL;
+    return ncp * 32 + G * (size_t)ns * (ncp * 16 + 8) + G * 2 * (size_t)R * (4 + 8);
+}
+
+template <int MODE, int R, int CPL>
+sq_status launch_row_quant_ring_inst(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
+                                     float* scale, cudaStream_t st, float eps, float* r_out, int ns) {
+    static bool attr_done[64] = {};
+    const DeviceInfo& di = device_info();
+    auto kern = row_quant_ring_kernel<MODE, R, CPL>;
+    if (!attr_done[di.device & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row_quant_ring_kernel)");
+        attr_done[di.device & 63] = true;
+    }
+    constexpr int G = kRingThreads / (32 * R);
+    const int64_t need = (rows + G - 1) / G;
+    const int grid = (int)(need < di.sm_count ? need : di.sm_count);
+    return launch_pdl("row_quant_ring_kernel", kern, dim3(grid), dim3(kRingThreads), ring_smem_bytes(R, CPL, ns), st,
+                      1, static_cast<const __nv_bfloat16*>(in), rows, K, s, q, scale, eps, r_out, ns,
+                      wait_limit_cycles());
+}
+
+template <int MODE, int R>
+sq_status launch_row_quant_ring_r(int cpl, const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
+                                  float* scale, cudaStream_t st, float eps, float* r_out, int ns) {
+    switch (cpl) {
+        case 5: return launch_row_quant_ring_inst<MODE, R, 5>(in, rows, K, s, q, scale, st, eps, r_out, ns);
+        case 6: return launch_row_quant_ring_inst<MODE, R, 6>(in, rows, K, s, q, scale, st, eps, r_out, ns);
+        case 7: return launch_row_quant_ring_inst<MODE, R, 7>(in, rows, K, s, q, scale, st, eps, r_out, ns);
+        default: return launch_row_quant_ring_inst<MODE, R, 8>(in, rows, K, s, q, scale, st, eps, r_out, ns);
+    }
+}
+
+// bf16 rows of 2064..16384 elements go to the streamed kernel: the fewest
+// warps per row (R = 2, 4 or 8) whose lanes hold the row in at most 8 chunks
+// each (CPL = 5..8 of them, the row padded to 32 * R * CPL chunks), and two
+// ring slots per group (one row in flight while one is processed: measured
+// faster than three or four). Returns false when K is outside that range.
+template <int MODE>
+bool launch_row_quant_ring(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q, float* scale,
+                           cudaStream_t st, float eps, float* r_out, sq_status& result) {
+    const int64_t nchunks = K / 8;
+    if (K <= 2048 || nchunks > (int64_t)32 * 8 * kRingCPL) return false;
+    const int R = nchunks <= (int64_t)32 * 2 * kRingCPL ? 2 : (nchunks <= (int64_t)32 * 4 * kRingCPL ? 4 : 8);
+    int cpl = (int)((nchunks + 32 * R - 1) / (32 * R));
+    if (cpl < 5) cpl = 5;
+    const int ns = 2;
+    if (ring_smem_bytes(R, cpl, ns) > kRingSmemMax) return false;
+    switch (R) {
+        case 2: result = launch_row_quant_ring_r<MODE, 2>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
+        case 4: result = launch_row_quant_ring_r<MODE, 4>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
+        default: result = launch_row_quant_ring_r<MODE, 8>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
+    }
+    return true;
+}
+
 template <typename T, int MODE>
 sq_status launch_row_quant(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
                            float* scale, cudaStream_t st, float eps = 0.0f, float* r_out = nullptr) {
     constexpr int CPL = RowFastCPL<T>::value;
     const int64_t nchunks = K / 8;
+    if constexpr (sizeof(T) == 2) {
+        sq_status res = SQ_OK;
+        if (launch_row_quant_ring<MODE>(in, rows, K, s, q, scale, st, eps, r_out, res)) return res;
+    }
     // the fewest warps per row whose lanes hold the row in CPL chunks each
     if (K <= kFastMaxK) {
         for (int R = 1; R <= 16; R *= 2) {
