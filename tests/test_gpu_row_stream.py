@@ -1,9 +1,9 @@
-"""The streamed row kernel (bf16 rows of 2064 to 16384 channels, staged in
+"""The streamed row kernel (bf16 rows of 2064 to 28672 channels, staged in
 shared memory by bulk copies): fold + quantize (a3), smooth + quantize (a4) and
 RMSNorm + quantize against the CPU oracle, through the C ABI.
 
 Bar: codes and scales bit-exact. The shapes cover every group width the kernel
-uses (2, 4 and 8 warps per row) and every chunk count per lane (5 to 8), rows
+uses (2, 4, 8 and 16 warps per row) and every chunk count per lane (5 to 8), rows
 padded to whole lanes and rows that fill them exactly, and many rows per
 group (the ring of row slots wraps many times); the
 special rows drive its exact paths: near-ties of the fast quotient, many
@@ -29,9 +29,10 @@ BF16 = torch.bfloat16
 
 # (rows, K) -> warps per row, chunks per lane (padded chunks): 2064 -> 2, 5 (62);
 # 4096 -> 2, 8; 4112 -> 4, 5 (126); 6144 -> 4, 6; 6160 -> 4, 7 (126); 8192 -> 4, 8;
-# 11008 -> 8, 6 (160); 12304 -> 8, 7 (254); 16384 -> 8, 8.
+# 11008 -> 8, 6 (160); 12304 -> 8, 7 (254); 16384 -> 8, 8; 16400 -> 16, 5 (510);
+# 28672 -> 16, 7.
 SHAPES = [(1, 2064), (37, 4096), (2500, 4096), (300, 4112), (17, 6144), (9, 6160), (200, 8192), (33, 11008),
-          (5, 12304), (3, 16384), (70, 16384)]
+          (5, 12304), (3, 16384), (70, 16384), (6, 16400), (300, 28672)]
 
 
 def dev(t):
@@ -113,7 +114,7 @@ def _tie_targets(scale):
     return np.array(out, np.float32)
 
 
-@pytest.mark.parametrize("K", [4096, 8192, 16384])
+@pytest.mark.parametrize("K", [4096, 8192, 16384, 28672])
 def test_near_ties(K):
     """With x = 1 the folded value is s itself and the smoothed value RN(1/s):
     choosing s puts hundreds of quotients within a few ulps of k + 1/2, in

@@ -743,7 +743,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
 }
 
 // ============================================================== the streamed row kernel (bf16)
-// bf16 rows of 2064 to 16384 elements. One CTA of 16 warps per SM, in groups
+// bf16 rows of 2064 to 28672 elements. One CTA of 16 warps per SM, in groups
 // of R warps; a group quantizes one row at a time, lane l of the group owning
 // the 8-element chunks l, l + 32R, ... (CPL of them: the row is padded with
 // zeros to 32 R CPL chunks, so the unrolled loops need no bounds checks and
@@ -1020,9 +1020,9 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         const float r = __frcp_rn(scale);
         const uint64_t r2 = f2_pack(r, r);
         uint32_t ntm = 0;
+        uint2 codes[CPL];
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
-            const int c = gl + i * 32 * R;
             {
                 uint32_t t[8];
                 float dm = 0.0f;
@@ -1037,12 +1037,16 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                     t[2 * p + 1] = __float_as_uint(t1);
                     dm = fmax3(dm, fabsf(d0), fabsf(d1));
                 }
-                uint2 codes;
-                codes.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-                codes.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
-                if (c < nch) *reinterpret_cast<uint2*>(rq + c * 8) = codes;
+                codes[i].x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+                codes[i].y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
                 ntm |= (dm >= 0.5f - kTieGuard ? 1u : 0u) << i;   // (padding: d = 0)
             }
+        }
+        // the stores apart from the arithmetic, which stays free of branches
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = gl + i * 32 * R;
+            if (c < nch) *reinterpret_cast<uint2*>(rq + c * 8) = codes[i];
         }
         if (gl == 0) scale_out[row] = scale;
         // near ties: the same fast quotient recomputed per element; those
@@ -1195,17 +1199,20 @@ sq_status launch_row_quant_ring_r(int cpl, const void* in, int64_t rows, int64_t
     }
 }
 
-// bf16 rows of 2064..16384 elements go to the streamed kernel: the fewest
-// warps per row (R = 2, 4 or 8) whose lanes hold the row in at most 8 chunks
+// bf16 rows of 2064..28672 elements go to the streamed kernel: the fewest
+// warps per row (R = 2, 4, 8 or 16) whose lanes hold the row in at most 8 chunks
 // each (CPL = 5..8 of them, the row padded to 32 * R * CPL chunks), and two
 // ring slots per group (one row in flight while one is processed: measured
-// faster than three or four). Returns false when K is outside that range.
+// faster than three or four). Returns false when K is outside that range or
+// the padded row, its multipliers and two slots exceed the shared memory of a
+// CTA (K above 28672).
 template <int MODE>
 bool launch_row_quant_ring(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q, float* scale,
                            cudaStream_t st, float eps, float* r_out, sq_status& result) {
     const int64_t nchunks = K / 8;
-    if (K <= 2048 || nchunks > (int64_t)32 * 8 * kRingCPL) return false;
-    const int R = nchunks <= (int64_t)32 * 2 * kRingCPL ? 2 : (nchunks <= (int64_t)32 * 4 * kRingCPL ? 4 : 8);
+    if (K <= 2048 || nchunks > (int64_t)32 * 16 * kRingCPL) return false;
+    int R = 2;
+    while ((int64_t)32 * R * kRingCPL < nchunks) R *= 2;
     int cpl = (int)((nchunks + 32 * R - 1) / (32 * R));
     if (cpl < 5) cpl = 5;
     const int ns = 2;
@@ -1213,7 +1220,8 @@ bool launch_row_quant_ring(const void* in, int64_t rows, int64_t K, const float*
     switch (R) {
         case 2: result = launch_row_quant_ring_r<MODE, 2>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
         case 4: result = launch_row_quant_ring_r<MODE, 4>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
-        default: result = launch_row_quant_ring_r<MODE, 8>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
+        case 8: result = launch_row_quant_ring_r<MODE, 8>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
+        default: result = launch_row_quant_ring_r<MODE, 16>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
     }
     return true;
 }
