@@ -814,7 +814,7 @@ __device__ __forceinline__ bool group_all(bool ok, int grp) {
     return r != 0;
 }
 
-template <int MODE, int R, int CPL>
+template <int MODE, int R, int CPL, bool FULL>
 __global__ void __launch_bounds__(kRingThreads, 1)
 row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
                       int8_t* __restrict__ q, float* __restrict__ scale_out, float eps, float* __restrict__ r_out,
@@ -824,7 +824,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
     constexpr uint32_t SLOT = NCP * 16u;         // bytes of one ring slot
     extern __shared__ __align__(128) uint8_t ring_smem[];
     const int64_t nchunks = K >> 3;
-    const int nch = (int)nchunks;
+    const int nch = FULL ? NCP : (int)nchunks;   // FULL: the row fills every lane's CPL chunks
     const uint32_t row_bytes = (uint32_t)K * 2u;
     float* mul_lo = reinterpret_cast<float*>(ring_smem);         // [NCP][4]: m_j of elements 0..3
     float* mul_hi = mul_lo + NCP * 4;                            // [NCP][4]: elements 4..7
@@ -1046,7 +1046,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
             const int c = gl + i * 32 * R;
-            if (c < nch) *reinterpret_cast<uint2*>(rq + c * 8) = codes[i];
+            if (FULL || c < nch) *reinterpret_cast<uint2*>(rq + c * 8) = codes[i];
         }
         if (gl == 0) scale_out[row] = scale;
         // near ties: the same fast quotient recomputed per element; those
@@ -1169,12 +1169,12 @@ size_t ring_smem_bytes(int R, int CPL, int ns) {
     return ncp * 32 + G * (size_t)ns * (ncp * 16 + 8) + G * 2 * (size_t)R * (4 + 8);
 }
 
-template <int MODE, int R, int CPL>
+template <int MODE, int R, int CPL, bool FULL>
 sq_status launch_row_quant_ring_inst(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
                                      float* scale, cudaStream_t st, float eps, float* r_out, int ns) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
-    auto kern = row_quant_ring_kernel<MODE, R, CPL>;
+    auto kern = row_quant_ring_kernel<MODE, R, CPL, FULL>;
     if (!attr_done[di.device & 63]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row_quant_ring_kernel)");
@@ -1191,12 +1191,18 @@ sq_status launch_row_quant_ring_inst(const void* in, int64_t rows, int64_t K, co
 template <int MODE, int R>
 sq_status launch_row_quant_ring_r(int cpl, const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
                                   float* scale, cudaStream_t st, float eps, float* r_out, int ns) {
+    // rows that fill every lane (K = 256 R CPL) drop the stores' bounds checks
+    const bool full = K / 8 == (int64_t)32 * R * cpl;
+#define SQ_RING_CPL(C)                                                                                   \
+    return full ? launch_row_quant_ring_inst<MODE, R, C, true>(in, rows, K, s, q, scale, st, eps, r_out, ns) \
+                : launch_row_quant_ring_inst<MODE, R, C, false>(in, rows, K, s, q, scale, st, eps, r_out, ns)
     switch (cpl) {
-        case 5: return launch_row_quant_ring_inst<MODE, R, 5>(in, rows, K, s, q, scale, st, eps, r_out, ns);
-        case 6: return launch_row_quant_ring_inst<MODE, R, 6>(in, rows, K, s, q, scale, st, eps, r_out, ns);
-        case 7: return launch_row_quant_ring_inst<MODE, R, 7>(in, rows, K, s, q, scale, st, eps, r_out, ns);
-        default: return launch_row_quant_ring_inst<MODE, R, 8>(in, rows, K, s, q, scale, st, eps, r_out, ns);
+        case 5: SQ_RING_CPL(5);
+        case 6: SQ_RING_CPL(6);
+        case 7: SQ_RING_CPL(7);
+        default: SQ_RING_CPL(8);
     }
+#undef SQ_RING_CPL
 }
 
 // bf16 rows of 2064..28672 elements go to the streamed kernel: the fewest
