@@ -138,6 +138,18 @@ sq_status sq_smooth_quant_act(const void* x, sq_dtype dt, int64_t T, int64_t K,
 sq_status sq_calibrate_absmax_pair(const void* x, int64_t T, const void* w, int64_t N, sq_dtype dt,
                                    int64_t K, float* xmax, float* wmax, sq_stream_t stream);
 
+/* ---------------------------------------------------------------- both quantizations in one launch
+ * sq_fold_smooth_quant_pair: step a3 on the weights w [N x K] (into wq,
+ * w_scale) and step a4 on the activations x [T x K] (into xq, x_scale) with the
+ * same smoothing factors s, in one launch where the library's streamed row
+ * kernel takes both tensors (bf16 inputs and K within its range), else as the
+ * two calls one after the other. Same results as sq_fold_quant_weights
+ * followed by sq_smooth_quant_act, bit for bit; same arguments and layouts as
+ * those two calls. Same dtype for both inputs. */
+sq_status sq_fold_smooth_quant_pair(const void* w, int64_t N, const void* x, int64_t T, sq_dtype dt, int64_t K,
+                                    const float* s, int8_t* wq, float* w_scale, int8_t* xq, float* x_scale,
+                                    sq_stream_t stream);
+
 /* ---------------------------------------------------------------- per-tensor scales (O2, O3)
  * One activation scale for the whole tensor instead of one per token: the
  * per-tensor dynamic (O2) and per-tensor static (O3) levels of "SmoothQuant

@@ -185,3 +185,55 @@ def test_keep_mask_fold_is_the_bulk_quantizer():
     oq, osc = oracle.quant_bulk(synth.host_array(x), keep)
     assert_equal(host(q), oq, "bulk codes")
     assert_bitexact_f32(host(sc), osc, "bulk scales")
+
+
+PAIR_SHAPES = [(300, 37, 4096), (1000, 7, 4112), (64, 200, 6160), (5, 900, 4096), (50, 3, 16384), (9, 5, 28672),
+               (40, 33, 2048)]
+
+
+@pytest.mark.parametrize("dtype", [BF16, torch.float32])
+@pytest.mark.parametrize("N,T,K", PAIR_SHAPES)
+def test_pair_launch_equals_the_two_calls(dtype, N, T, K):
+    """a3 and a4 in one launch (weights' rows, then activations' rows): the
+    same codes and scales as the two calls and as the oracle. K = 28672 (two
+    multiplier tables do not fit beside the ring) and K = 2048 or fp32 rows
+    (outside the streamed kernel) take the two calls."""
+    g = torch.Generator().manual_seed(N + T + K)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(dtype)
+    x = outlier_x(T, K, seed=N * 7 + K).to(dtype)
+    if N > 2:
+        w[1] = 0
+    if T > 2:
+        x[2] = 0
+        x[1] *= 1e-35
+    s = s_for(K, K + 3)
+    sd = dev(torch.from_numpy(s))
+    wd, xd = dev(w), dev(x)
+    wq, wsc, xq, xsc = sq.sq_fold_smooth_quant_pair(wd, xd, sd)
+    wq1, wsc1 = sq.sq_fold_quant_weights(wd, sd)
+    xq1, xsc1 = sq.sq_smooth_quant_act(xd, sd)
+    assert_equal(host(wq), host(wq1), "pair vs separate: wq")
+    assert_equal(host(xq), host(xq1), "pair vs separate: xq")
+    assert_bitexact_f32(host(wsc), host(wsc1), "pair vs separate: w_scale")
+    assert_bitexact_f32(host(xsc), host(xsc1), "pair vs separate: x_scale")
+    oq, osc = oracle.fold_quant_weights(synth.host_array(w), s)
+    assert_equal(host(wq), oq, "pair wq vs oracle")
+    assert_bitexact_f32(host(wsc), osc, "pair w_scale vs oracle")
+    oq, osc = oracle.smooth_quant_act(synth.host_array(x), s)
+    assert_equal(host(xq), oq, "pair xq vs oracle")
+    assert_bitexact_f32(host(xsc), osc, "pair x_scale vs oracle")
+    assert sq.sq_get_status() == sq.SQ_OK
+
+
+def test_pair_launch_qkv_prefill_7b_full_size():
+    wl = synth.WORKLOADS["qkv_prefill_7b"]
+    x, w = synth.make(wl.name)
+    hx, hw = synth.host_array(x), synth.host_array(w)
+    s = oracle.smooth_factors(oracle.col_absmax(hx), oracle.col_absmax(hw), wl.alpha)
+    wq, wsc, xq, xsc = sq.sq_fold_smooth_quant_pair(dev(w), dev(x), dev(torch.from_numpy(s)))
+    oq, osc = oracle.fold_quant_weights(hw, s)
+    assert_equal(host(wq), oq, "full-size pair wq")
+    assert_bitexact_f32(host(wsc), osc, "full-size pair w_scale")
+    oq, osc = oracle.smooth_quant_act(hx, s)
+    assert_equal(host(xq), oq, "full-size pair xq")
+    assert_bitexact_f32(host(xsc), osc, "full-size pair x_scale")

@@ -157,6 +157,8 @@ sq_status fold_quant_weights_impl(const void*, sq_dtype, int64_t, int64_t, const
                                   cudaStream_t);
 sq_status smooth_quant_act_impl(const void*, sq_dtype, int64_t, int64_t, const float*, int8_t*, float*,
                                 cudaStream_t);
+sq_status fold_smooth_quant_pair_impl(const void*, int64_t, const void*, int64_t, sq_dtype, int64_t, const float*,
+                                      int8_t*, float*, int8_t*, float*, cudaStream_t);
 sq_status calibrate_absmax_pair_impl(const void*, int64_t, const void*, int64_t, sq_dtype, int64_t, float*, float*,
                                      cudaStream_t);
 
@@ -218,8 +220,7 @@ sq_status linear_impl(const void* x, const void* w, sq_dtype in_dt, int64_t M, i
     sq_status r;
     if ((r = calibrate_absmax_pair_impl(xd, M, wd, N, in_dt, K, xmax, wmax, st)) != SQ_OK) return r;
     if ((r = smooth_factors_impl(xmax, wmax, K, alpha, eps, s, st)) != SQ_OK) return r;
-    if ((r = fold_quant_weights_impl(wd, in_dt, N, K, s, wq, wsc, st)) != SQ_OK) return r;
-    if ((r = smooth_quant_act_impl(xd, in_dt, M, K, s, xq, xs, st)) != SQ_OK) return r;
+    if ((r = fold_smooth_quant_pair_impl(wd, N, xd, M, in_dt, K, s, wq, wsc, xq, xs, st)) != SQ_OK) return r;
     if ((x_host || w_host) && (e = cudaEventRecord(cs.inputs_free, st)) != cudaSuccess)
         return cuda_fail(e, "record the end of the staged inputs' use");
     if ((r = gemm_dispatch(xq, xs, wq, wsc, M, N, K, yd, out_dt, base + L.gemm_ws, L.gemm_ws_bytes, st)) != SQ_OK)

@@ -814,11 +814,21 @@ __device__ __forceinline__ bool group_all(bool ok, int grp) {
     return r != 0;
 }
 
-template <int MODE, int R, int CPL, bool FULL>
+// The second tensor of a pair launch (the activations, smoothed), quantized in
+// the same launch as the weights: its rows follow the first tensor's.
+struct RingPair {
+    const __nv_bfloat16* in2 = nullptr;
+    int64_t rows2 = 0;
+    int8_t* q2 = nullptr;
+    float* scale2 = nullptr;
+};
+
+template <int MODE, int R, int CPL, bool FULL, bool PAIR>
 __global__ void __launch_bounds__(kRingThreads, 1)
 row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
                       int8_t* __restrict__ q, float* __restrict__ scale_out, float eps, float* __restrict__ r_out,
-                      int ns, long long wait_limit) {
+                      int ns, long long wait_limit, RingPair pr) {
+    static_assert(!PAIR || MODE == kFold, "the pair launch folds its first tensor and smooths its second");
     constexpr int G = kRingThreads / (32 * R);   // groups per CTA
     constexpr int NCP = 32 * R * CPL;            // chunks of a row padded to whole lanes
     constexpr uint32_t SLOT = NCP * 16u;         // bytes of one ring slot
@@ -828,7 +838,9 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
     const uint32_t row_bytes = (uint32_t)K * 2u;
     float* mul_lo = reinterpret_cast<float*>(ring_smem);         // [NCP][4]: m_j of elements 0..3
     float* mul_hi = mul_lo + NCP * 4;                            // [NCP][4]: elements 4..7
-    uint8_t* slots = ring_smem + NCP * 32;                       // [G][ns][SLOT]
+    float* mul2_lo = mul_hi + NCP * 4;                           // PAIR: RN(1/s_j) for the second tensor
+    float* mul2_hi = mul2_lo + NCP * 4;
+    uint8_t* slots = ring_smem + NCP * (PAIR ? 64 : 32);         // [G][ns][SLOT]
     uint64_t* bars = reinterpret_cast<uint64_t*>(slots + (size_t)G * ns * SLOT);   // [G][ns]
     float* red = reinterpret_cast<float*>(bars + G * ns);        // [G][2][R]
     double* red64 = reinterpret_cast<double*>(red + G * 2 * R);  // [G][2][R]
@@ -850,14 +862,19 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
     pdl_wait();
     pdl_trigger();
 
+    // rows [0, rows) of the first tensor, then (PAIR) rows [rows, total) of the second
+    const int64_t total = rows + (PAIR ? pr.rows2 : 0);
+    auto row_src = [&](int64_t g) {
+        return (PAIR && g >= rows) ? pr.in2 + (g - rows) * K : in + g * K;
+    };
     const int64_t stride = (int64_t)gridDim.x * G;
     const int64_t row0 = (int64_t)blockIdx.x * G + grp;
     if (gl == 0) {
         for (int j = 0; j < ns; ++j) {
             const int64_t row = row0 + (int64_t)j * stride;
-            if (row < rows) {
+            if (row < total) {
                 mbar_arrive_expect_tx(bar0 + 8u * j, row_bytes);
-                bulk_copy_g2s(smem_u32(my_slots + (size_t)j * SLOT), in + row * K, row_bytes, bar0 + 8u * j);
+                bulk_copy_g2s(smem_u32(my_slots + (size_t)j * SLOT), row_src(row), row_bytes, bar0 + 8u * j);
             }
         }
     }
@@ -876,6 +893,14 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         }
         *reinterpret_cast<float4*>(mul_lo + c * 4) = a;
         *reinterpret_cast<float4*>(mul_hi + c * 4) = b;
+        if (PAIR) {
+            if (c < nch) {
+                a = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
+                b = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
+            }
+            *reinterpret_cast<float4*>(mul2_lo + c * 4) = a;
+            *reinterpret_cast<float4*>(mul2_hi + c * 4) = b;
+        }
     }
     {
         const int tail = (int)((SLOT - row_bytes) / 16u);
@@ -890,7 +915,15 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
     int it = 0, sl = 0, ps = ns - 1;   // iteration, its slot, the previous iteration's slot
     uint32_t parity = 0;
     bool failed = false;
-    for (int64_t row = row0; row < rows; row += stride, ++it) {
+    for (int64_t g = row0; g < total; g += stride, ++it) {
+        // this row's tensor: the first (MODE), or the second (smoothed) of a pair
+        const bool second = PAIR && g >= rows;
+        const bool smooth = MODE == kSmooth || second;
+        const int64_t row = second ? g - rows : g;
+        int8_t* const qo = second ? pr.q2 : q;
+        float* const so = second ? pr.scale2 : scale_out;
+        const float* const mlo = second ? mul2_lo : mul_lo;
+        const float* const mhi = second ? mul2_hi : mul_hi;
         const bool ok = mbar_wait_sleep(bar0 + 8u * sl, parity, wait_limit, &abort_sh, SITE_QUANT_WAIT);
         __syncwarp();   // the barrier below is warp-aligned
         if (!group_all<R>(ok, grp)) {
@@ -899,10 +932,10 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         }
         // every warp of the group is done with the previous row's slot: refill it
         if (it > 0 && gl == 0) {
-            const int64_t nr = row + (int64_t)(ns - 1) * stride;
-            if (nr < rows) {
+            const int64_t nr = g + (int64_t)(ns - 1) * stride;
+            if (nr < total) {
                 mbar_arrive_expect_tx(bar0 + 8u * ps, row_bytes);
-                bulk_copy_g2s(smem_u32(my_slots + (size_t)ps * SLOT), in + nr * K, row_bytes, bar0 + 8u * ps);
+                bulk_copy_g2s(smem_u32(my_slots + (size_t)ps * SLOT), row_src(nr), row_bytes, bar0 + 8u * ps);
             }
         }
         const uint8_t* src = my_slots + (size_t)sl * SLOT;
@@ -941,8 +974,8 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         for (int i = 0; i < CPL; ++i) {
             const int c = gl + i * 32 * R;
             const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-            const float4 a = *reinterpret_cast<const float4*>(mul_lo + c * 4);
-            const float4 b = *reinterpret_cast<const float4*>(mul_hi + c * 4);
+            const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
+            const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
             const uint64_t mp[4] = {f2_pack(a.x, a.y), f2_pack(a.z, a.w), f2_pack(b.x, b.y), f2_pack(b.z, b.w)};
             float cmax = 0.0f;
 #pragma unroll
@@ -959,7 +992,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         }
         float amax = group_max<R>(m, red, grp, wig, lane, bank);
         bank ^= 1;
-        int8_t* rq = q + row * K;
+        int8_t* rq = qo + row * K;
 
         if (!(amax >= kSmallRow)) {
             // zero, tiny or near-underflow row: exact maximum and codes
@@ -970,7 +1003,8 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                 if (c < nch) {
                     RawChunk<__nv_bfloat16> ch;
                     ch.a = *reinterpret_cast<const uint4*>(src + c * 16);
-                    ex = fmaxf(ex, exact_chunk_max_in<__nv_bfloat16, MODE>(ch, s + c * 8, rn));
+                    ex = fmaxf(ex, second ? exact_chunk_max_in<__nv_bfloat16, kSmooth>(ch, s + c * 8, rn)
+                                          : exact_chunk_max_in<__nv_bfloat16, MODE>(ch, s + c * 8, rn));
                 }
             }
             const float a = group_max<R>(ex, red, grp, wig, lane, bank);
@@ -983,14 +1017,15 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                     RawChunk<__nv_bfloat16> ch;
                     ch.a = *reinterpret_cast<const uint4*>(src + c * 16);
                     *reinterpret_cast<uint2*>(rq + c * 8) =
-                        exact_chunk_codes_in<__nv_bfloat16, MODE>(ch, s + c * 8, scale, rn, a == 0.0f);
+                        second ? exact_chunk_codes_in<__nv_bfloat16, kSmooth>(ch, s + c * 8, scale, rn, a == 0.0f)
+                               : exact_chunk_codes_in<__nv_bfloat16, MODE>(ch, s + c * 8, scale, rn, a == 0.0f);
                 }
             }
-            if (gl == 0) scale_out[row] = scale;
+            if (gl == 0) so[row] = scale;
             continue;
         }
 
-        if (MODE == kSmooth) {
+        if (smooth) {
             // exact values of the candidates (normally the maximum alone)
             const float thr = __fmul_rn(amax, kRingCandidate);
             uint32_t cand = 0;
@@ -1002,13 +1037,13 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                 cand &= cand - 1;
                 const int c = gl + i * 32 * R;
                 const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-                const float4 a = *reinterpret_cast<const float4*>(mul_lo + c * 4);
-                const float4 b = *reinterpret_cast<const float4*>(mul_hi + c * 4);
+                const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
+                const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
                 const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float x = bf16_elem(w, e);
-                    if (fabsf(__fmul_rn(x, mv[e])) >= thr) ex = fmaxf(ex, exact_abs<MODE>(x, __ldg(s + c * 8 + e), rn));
+                    if (fabsf(__fmul_rn(x, mv[e])) >= thr) ex = fmaxf(ex, exact_abs<kSmooth>(x, __ldg(s + c * 8 + e), rn));
                 }
             }
             amax = group_max<R>(ex, red, grp, wig, lane, bank);
@@ -1048,7 +1083,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             const int c = gl + i * 32 * R;
             if (FULL || c < nch) *reinterpret_cast<uint2*>(rq + c * 8) = codes[i];
         }
-        if (gl == 0) scale_out[row] = scale;
+        if (gl == 0) so[row] = scale;
         // near ties: the same fast quotient recomputed per element; those
         // within the guard get the IEEE-division code (same thread, later store)
         while (ntm) {
@@ -1056,8 +1091,8 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             ntm &= ntm - 1;
             const int c = gl + i * 32 * R;
             const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-            const float4 a = *reinterpret_cast<const float4*>(mul_lo + c * 4);
-            const float4 b = *reinterpret_cast<const float4*>(mul_hi + c * 4);
+            const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
+            const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
             const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -1066,7 +1101,8 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                 const float tf = __fmaf_rn(vf, r, kMagic);
                 const float df = __fmaf_rn(vf, r, __fsub_rn(kMagic, tf));
                 if (fabsf(df) >= 0.5f - kTieGuard)
-                    rq[c * 8 + e] = (int8_t)exact_code<MODE>(x, __ldg(s + c * 8 + e), scale, rn);
+                    rq[c * 8 + e] = (int8_t)(second ? exact_code<kSmooth>(x, __ldg(s + c * 8 + e), scale, rn)
+                                                    : exact_code<MODE>(x, __ldg(s + c * 8 + e), scale, rn));
             }
         }
     }
@@ -1076,7 +1112,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         // before the CTA exits (bounded)
         for (int j = it; j < it + ns - 1; ++j) {
             const int64_t row = row0 + (int64_t)j * stride;
-            if (row < rows) mbar_wait(bar0 + 8u * (j % ns), (uint32_t)(j / ns) & 1u, wait_limit, &never_sh, SITE_QUANT_DRAIN);
+            if (row < total) mbar_wait(bar0 + 8u * (j % ns), (uint32_t)(j / ns) & 1u, wait_limit, &never_sh, SITE_QUANT_DRAIN);
         }
     }
 }
@@ -1160,42 +1196,45 @@ sq_status launch_row_quant_fast_inst(const void* in, int64_t rows, int64_t K, co
                       static_cast<const T*>(in), rows, K, s, q, scale, eps, r_out);
 }
 
-// The streamed kernel's shared memory: multipliers and ns row slots per group,
-// both padded to 32 * R * CPL chunks, the slots' mbarriers and the group
-// reduction slots.
-size_t ring_smem_bytes(int R, int CPL, int ns) {
+// The streamed kernel's shared memory: multipliers (two tables for a pair
+// launch) and ns row slots per group, both padded to 32 * R * CPL chunks, the
+// slots' mbarriers and the group reduction slots.
+size_t ring_smem_bytes(int R, int CPL, int ns, bool pair) {
     const size_t G = (size_t)(kRingThreads / (32 * R));
     const size_t ncp = (size_t)32 * R * CPL;
-    return ncp * 32 + G * (size_t)ns * (ncp * 16 + 8) + G * 2 * (size_t)R * (4 + 8);
+    return ncp * (pair ? 64 : 32) + G * (size_t)ns * (ncp * 16 + 8) + G * 2 * (size_t)R * (4 + 8);
 }
 
-template <int MODE, int R, int CPL, bool FULL>
+template <int MODE, int R, int CPL, bool FULL, bool PAIR>
 sq_status launch_row_quant_ring_inst(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
-                                     float* scale, cudaStream_t st, float eps, float* r_out, int ns) {
+                                     float* scale, cudaStream_t st, float eps, float* r_out, int ns,
+                                     const RingPair& pr) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
-    auto kern = row_quant_ring_kernel<MODE, R, CPL, FULL>;
+    auto kern = row_quant_ring_kernel<MODE, R, CPL, FULL, PAIR>;
     if (!attr_done[di.device & 63]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row_quant_ring_kernel)");
         attr_done[di.device & 63] = true;
     }
     constexpr int G = kRingThreads / (32 * R);
-    const int64_t need = (rows + G - 1) / G;
+    const int64_t need = (rows + (PAIR ? pr.rows2 : 0) + G - 1) / G;
     const int grid = (int)(need < di.sm_count ? need : di.sm_count);
-    return launch_pdl("row_quant_ring_kernel", kern, dim3(grid), dim3(kRingThreads), ring_smem_bytes(R, CPL, ns), st,
-                      1, static_cast<const __nv_bfloat16*>(in), rows, K, s, q, scale, eps, r_out, ns,
-                      wait_limit_cycles());
+    return launch_pdl("row_quant_ring_kernel", kern, dim3(grid), dim3(kRingThreads), ring_smem_bytes(R, CPL, ns, PAIR),
+                      st, 1, static_cast<const __nv_bfloat16*>(in), rows, K, s, q, scale, eps, r_out, ns,
+                      wait_limit_cycles(), pr);
 }
 
-template <int MODE, int R>
+template <int MODE, int R, bool PAIR>
 sq_status launch_row_quant_ring_r(int cpl, const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
-                                  float* scale, cudaStream_t st, float eps, float* r_out, int ns) {
+                                  float* scale, cudaStream_t st, float eps, float* r_out, int ns,
+                                  const RingPair& pr) {
     // rows that fill every lane (K = 256 R CPL) drop the stores' bounds checks
     const bool full = K / 8 == (int64_t)32 * R * cpl;
-#define SQ_RING_CPL(C)                                                                                   \
-    return full ? launch_row_quant_ring_inst<MODE, R, C, true>(in, rows, K, s, q, scale, st, eps, r_out, ns) \
-                : launch_row_quant_ring_inst<MODE, R, C, false>(in, rows, K, s, q, scale, st, eps, r_out, ns)
+#define SQ_RING_CPL(C)                                                                                          \
+    return full ? launch_row_quant_ring_inst<MODE, R, C, true, PAIR>(in, rows, K, s, q, scale, st, eps, r_out, ns, \
+                                                                     pr)                                          \
+                : launch_row_quant_ring_inst<MODE, R, C, false, PAIR>(in, rows, K, s, q, scale, st, eps, r_out, ns, pr)
     switch (cpl) {
         case 5: SQ_RING_CPL(5);
         case 6: SQ_RING_CPL(6);
@@ -1212,9 +1251,10 @@ sq_status launch_row_quant_ring_r(int cpl, const void* in, int64_t rows, int64_t
 // faster than three or four). Returns false when K is outside that range or
 // the padded row, its multipliers and two slots exceed the shared memory of a
 // CTA (K above 28672).
-template <int MODE>
+template <int MODE, bool PAIR = false>
 bool launch_row_quant_ring(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q, float* scale,
-                           cudaStream_t st, float eps, float* r_out, sq_status& result) {
+                           cudaStream_t st, float eps, float* r_out, sq_status& result,
+                           const RingPair& pr = RingPair{}) {
     const int64_t nchunks = K / 8;
     if (K <= 2048 || nchunks > (int64_t)32 * 16 * kRingCPL) return false;
     int R = 2;
@@ -1222,12 +1262,12 @@ bool launch_row_quant_ring(const void* in, int64_t rows, int64_t K, const float*
     int cpl = (int)((nchunks + 32 * R - 1) / (32 * R));
     if (cpl < 5) cpl = 5;
     const int ns = 2;
-    if (ring_smem_bytes(R, cpl, ns) > kRingSmemMax) return false;
+    if (ring_smem_bytes(R, cpl, ns, PAIR) > kRingSmemMax) return false;
     switch (R) {
-        case 2: result = launch_row_quant_ring_r<MODE, 2>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
-        case 4: result = launch_row_quant_ring_r<MODE, 4>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
-        case 8: result = launch_row_quant_ring_r<MODE, 8>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
-        default: result = launch_row_quant_ring_r<MODE, 16>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns); break;
+        case 2: result = launch_row_quant_ring_r<MODE, 2, PAIR>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr); break;
+        case 4: result = launch_row_quant_ring_r<MODE, 4, PAIR>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr); break;
+        case 8: result = launch_row_quant_ring_r<MODE, 8, PAIR>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr); break;
+        default: result = launch_row_quant_ring_r<MODE, 16, PAIR>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr); break;
     }
     return true;
 }
@@ -1442,6 +1482,37 @@ sq_status smooth_quant_act_impl(const void* x, sq_dtype dt, int64_t T, int64_t K
     return row_quant_common(kSmooth, x, dt, T, K, s, xq, x_scale, st);
 }
 
+// a3 and a4 in one launch where the streamed kernel takes both (bf16, and the
+// two multiplier tables fit in shared memory beside the ring): the weights'
+// rows, then the activations'. Elsewhere the two calls, one after the other.
+sq_status fold_smooth_quant_pair_impl(const void* w, int64_t N, const void* x, int64_t T, sq_dtype dt, int64_t K,
+                                      const float* s, int8_t* wq, float* w_scale, int8_t* xq, float* x_scale,
+                                      cudaStream_t st) {
+    sq_status r;
+    if ((r = check_input_dtype(dt)) != SQ_OK) return r;
+    if ((r = check_matrix(w, N, K, "w")) != SQ_OK) return r;
+    if ((r = check_matrix(x, T, K, "x")) != SQ_OK) return r;
+    if (N == 0) return smooth_quant_act_impl(x, dt, T, K, s, xq, x_scale, st);
+    if (T == 0) return fold_quant_weights_impl(w, dt, N, K, s, wq, w_scale, st);
+    if (K == 0) { set_error("K must be positive"); return SQ_ERR_INVALID_ARG; }
+    if (!s || !wq || !w_scale || !xq || !x_scale) { set_error("NULL pointer"); return SQ_ERR_INVALID_ARG; }
+    if (!aligned16(s) || !aligned16(wq) || !aligned16(xq)) {
+        set_error("s and codes must be 16-byte aligned");
+        return SQ_ERR_UNSUPPORTED;
+    }
+    if (dt == SQ_BF16) {
+        RingPair pr;
+        pr.in2 = static_cast<const __nv_bfloat16*>(x);
+        pr.rows2 = T;
+        pr.q2 = xq;
+        pr.scale2 = x_scale;
+        sq_status res = SQ_OK;
+        if (launch_row_quant_ring<kFold, true>(w, N, K, s, wq, w_scale, st, 0.0f, nullptr, res, pr)) return res;
+    }
+    if ((r = fold_quant_weights_impl(w, dt, N, K, s, wq, w_scale, st)) != SQ_OK) return r;
+    return smooth_quant_act_impl(x, dt, T, K, s, xq, x_scale, st);
+}
+
 }  // namespace sq
 
 extern "C" {
@@ -1481,6 +1552,12 @@ sq_status sq_fold_quant_weights(const void* w, sq_dtype dt, int64_t N, int64_t K
 sq_status sq_smooth_quant_act(const void* x, sq_dtype dt, int64_t T, int64_t K, const float* s,
                               int8_t* xq, float* x_scale, sq_stream_t stream) {
     return sq::smooth_quant_act_impl(x, dt, T, K, s, xq, x_scale, (cudaStream_t)stream);
+}
+
+sq_status sq_fold_smooth_quant_pair(const void* w, int64_t N, const void* x, int64_t T, sq_dtype dt, int64_t K,
+                                    const float* s, int8_t* wq, float* w_scale, int8_t* xq, float* x_scale,
+                                    sq_stream_t stream) {
+    return sq::fold_smooth_quant_pair_impl(w, N, x, T, dt, K, s, wq, w_scale, xq, x_scale, (cudaStream_t)stream);
 }
 
 }  // extern "C"

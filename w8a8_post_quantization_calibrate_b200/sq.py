@@ -44,6 +44,7 @@ _SIGS = {
     "sq_fold_quant_weights": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_smooth_quant_act": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_calibrate_absmax_pair": ([_vp, _i64, _vp, _i64, _int, _i64, _vp, _vp, _vp], _int),
+    "sq_fold_smooth_quant_pair": ([_vp, _i64, _vp, _i64, _int, _i64, _vp, _vp, _vp, _vp, _vp, _vp], _int),
     "sq_fold_quant_weights_e4m3": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_smooth_quant_act_e4m3": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_w8a8_gemm_e4m3": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp], _int),
@@ -175,6 +176,28 @@ def sq_calibrate_absmax_pair(x: torch.Tensor, w: torch.Tensor, xmax: torch.Tenso
     _check(_lib.sq_calibrate_absmax_pair(_dev(x, "x"), T, _dev(w, "w"), N, _dt(x), K, _dev(xmax, "xmax"),
                                          _dev(wmax, "wmax"), _stream(stream)), "sq_calibrate_absmax_pair")
     return xmax, wmax
+
+
+def sq_fold_smooth_quant_pair(w: torch.Tensor, x: torch.Tensor, s: torch.Tensor, wq=None, w_scale=None, xq=None,
+                              x_scale=None, stream=None):
+    """a3 on w and a4 on x with the same s, in one launch where possible ->
+    (wq, w_scale, xq, x_scale)."""
+    N, K = w.shape
+    T = x.shape[0]
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must have the same dtype")
+    if wq is None:
+        wq = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=w.device)
+    if xq is None:
+        xq = torch.empty((T, K), dtype=torch.int8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(_lib.sq_fold_smooth_quant_pair(_dev(w, "w"), N, _dev(x, "x"), T, _dt(w), K, _dev(s, "s"), _dev(wq, "wq"),
+                                          _dev(w_scale, "w_scale"), _dev(xq, "xq"), _dev(x_scale, "x_scale"),
+                                          _stream(stream)), "sq_fold_smooth_quant_pair")
+    return wq, w_scale, xq, x_scale
 
 
 def sq_fold_quant_weights_e4m3(w: torch.Tensor, s: torch.Tensor, wq=None, w_scale=None, stream=None):
