@@ -3,7 +3,7 @@ shared memory by bulk copies): fold + quantize (a3), smooth + quantize (a4) and
 RMSNorm + quantize against the CPU oracle, through the C ABI.
 
 Bar: codes and scales bit-exact. The shapes cover every group width the kernel
-uses (2, 4, 8 and 16 warps per row) and every chunk count per lane (5 to 8), rows
+uses (2, 4, 8 and 16 warps per row) and every chunk count per lane (5 to 8, and 10), rows
 padded to whole lanes and rows that fill them exactly, and many rows per
 group (the ring of row slots wraps many times); the
 special rows drive its exact paths: near-ties of the fast quotient, many
@@ -28,11 +28,11 @@ DEV = torch.device("cuda", 0)
 BF16 = torch.bfloat16
 
 # (rows, K) -> warps per row, chunks per lane (padded chunks): 2064 -> 2, 5 (62);
-# 4096 -> 2, 8; 4112 -> 4, 5 (126); 6144 -> 4, 6; 6160 -> 4, 7 (126); 8192 -> 4, 8;
-# 11008 -> 8, 6 (160); 12304 -> 8, 7 (254); 16384 -> 8, 8; 16400 -> 16, 5 (510);
-# 28672 -> 16, 7.
-SHAPES = [(1, 2064), (37, 4096), (2500, 4096), (300, 4112), (17, 6144), (9, 6160), (200, 8192), (33, 11008),
-          (5, 12304), (3, 16384), (70, 16384), (6, 16400), (300, 28672)]
+# 4096 -> 2, 8; 4112 -> 2, 10 (126); 5120 -> 2, 10; 6144 -> 4, 6; 6160 -> 4, 7 (126);
+# 8192 -> 4, 8; 11008 -> 8, 6 (160); 12304 -> 8, 7 (254); 16384 -> 8, 8;
+# 16400 -> 16, 5 (510); 28672 -> 16, 7.
+SHAPES = [(1, 2064), (37, 4096), (2500, 4096), (300, 4112), (21, 5120), (17, 6144), (9, 6160), (200, 8192),
+          (33, 11008), (5, 12304), (3, 16384), (70, 16384), (6, 16400), (300, 28672)]
 
 
 def dev(t):
@@ -134,7 +134,7 @@ def test_near_ties(K):
     check_smooth(torch.ones(2, K, dtype=BF16), s_smooth, f"smooth near ties K={K}")
 
 
-@pytest.mark.parametrize("K", [4096, 6160, 16384])
+@pytest.mark.parametrize("K", [4096, 5120, 6160, 16384])
 def test_many_candidates_for_the_maximum(K):
     """Smoothed rows whose largest values differ by a few ulps, spread over
     all lanes and warps of the group: only exact divisions can tell them
@@ -187,8 +187,8 @@ def test_keep_mask_fold_is_the_bulk_quantizer():
     assert_bitexact_f32(host(sc), osc, "bulk scales")
 
 
-PAIR_SHAPES = [(300, 37, 4096), (1000, 7, 4112), (64, 200, 6160), (5, 900, 4096), (50, 3, 16384), (9, 5, 28672),
-               (40, 33, 2048)]
+PAIR_SHAPES = [(300, 37, 4096), (1000, 7, 4112), (70, 90, 5120), (64, 200, 6160), (5, 900, 4096), (50, 3, 16384),
+               (9, 5, 28672), (40, 33, 2048)]
 
 
 @pytest.mark.parametrize("dtype", [BF16, torch.float32])
