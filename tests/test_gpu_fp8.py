@@ -150,3 +150,71 @@ def test_e4m3_rejects_int32_output():
     with pytest.raises(sq.SqError) as e:
         sq.sq_w8a8_gemm_e4m3(xq, sc[:4], wq, sc, out_dtype=torch.int32)
     assert e.value.status == sq.SQ_ERR_UNSUPPORTED
+
+
+def _e4m3_midpoints():
+    """Every rounding boundary of E4M3 between its smallest subnormal and 448:
+    (k + 1/2) * quantum in each binade (quantum 2^-9 below 2^-6)."""
+    mids = [(k + 0.5) * 2.0 ** -9 for k in range(8)]
+    for e in range(-6, 9):
+        mids += [2.0 ** e * (1 + (k + 0.5) / 8) for k in range(8)]
+    return np.array([m for m in mids if m < 448.0])
+
+
+@pytest.mark.parametrize("K", [4096, 5120, 28672])
+def test_e4m3_stream_kernel_midpoints(K):
+    """Quotients at, and a few ulps either side of, every E4M3 rounding boundary
+    (subnormal band and saturation included), for the streamed kernel's fast
+    pass: with a power-of-two scale the quotient is exact, so exact ties occur.
+    x = 1 makes the folded value s itself and the smoothed value RN(1/s)."""
+    rng = np.random.default_rng(K)
+    scale = 0.125                                      # amax = 56 -> scale = 56 / 448
+    targets = []
+    for m in _e4m3_midpoints():
+        v0 = np.float32(m * scale)
+        for d in (-3, -1, 0, 1, 3):
+            targets.append(np.float32(v0 + d * np.spacing(v0)))
+    targets = np.array(targets, np.float32)
+    assert len(targets) < K - 1
+    s_fold = rng.uniform(0.01, 0.5, K).astype(np.float32)
+    s_fold[0] = 56.0
+    s_fold[rng.permutation(np.arange(1, K))[: len(targets)]] = targets
+    w = torch.ones(4, K, dtype=torch.bfloat16)
+    w[1] = -1.0
+    w[2, ::2] = 0.75                                   # scale 42 / 448, not a power of two
+    w[3] = -0.0                                        # all-zero row of negative zeros: codes 0x80, scale 1
+    hw = synth.host_array(w)
+    sd = dev(torch.from_numpy(s_fold))
+    q, sc = sq.sq_fold_quant_weights_e4m3(dev(w), sd)
+    oq, osc = oracle.fold_quant_weights_e4m3(hw, s_fold)
+    assert_equal(host(q), oq, "E4M3 fold codes at the boundaries")
+    assert_bitexact_f32(host(sc), osc, "E4M3 fold scales")
+    s_smooth = (np.float32(1.0) / s_fold).astype(np.float32)
+    x = torch.ones(3, K, dtype=torch.bfloat16)
+    x[1] = -1.0
+    x[2] = 0.0
+    q, sc = sq.sq_smooth_quant_act_e4m3(dev(x), dev(torch.from_numpy(s_smooth)))
+    oq, osc = oracle.smooth_quant_act_e4m3(synth.host_array(x), s_smooth)
+    assert_equal(host(q), oq, "E4M3 smooth codes at the boundaries")
+    assert_bitexact_f32(host(sc), osc, "E4M3 smooth scales")
+
+
+@pytest.mark.parametrize("K", [4096, 5120])
+def test_e4m3_stream_kernel_rows(K):
+    """Outlier rows, tiny rows (near the exact-path threshold) and many rows per
+    group through the streamed kernel's E4M3 pass."""
+    x = outlier_x(700, K, torch.bfloat16, seed=K + 11, n_out=4, scale=80.0)
+    x[3] *= 1e-30
+    x[4] *= 1e-36
+    x[5, 7] = 3e4
+    s = s_for(K, K + 5)
+    sd = dev(torch.from_numpy(s))
+    hx = synth.host_array(x)
+    q, sc = sq.sq_smooth_quant_act_e4m3(dev(x), sd)
+    oq, osc = oracle.smooth_quant_act_e4m3(hx, s)
+    assert_equal(host(q), oq, "E4M3 smooth codes")
+    assert_bitexact_f32(host(sc), osc, "E4M3 smooth scales")
+    q, sc = sq.sq_fold_quant_weights_e4m3(dev(x), sd)
+    oq, osc = oracle.fold_quant_weights_e4m3(hx, s)
+    assert_equal(host(q), oq, "E4M3 fold codes")
+    assert_bitexact_f32(host(sc), osc, "E4M3 fold scales")

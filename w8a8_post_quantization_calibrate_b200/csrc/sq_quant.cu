@@ -432,6 +432,13 @@ __device__ __noinline__ uint32_t exact_code(float x, float s_j, float scale, flo
     return (uint32_t)qi & 0xffu;
 }
 
+// The code of one element in either format (int8: as exact_code; E4M3: the
+// IEEE quotient converted with round-to-nearest-even and saturation).
+template <int MODE, int FMT>
+__device__ __noinline__ uint32_t exact_code_fmt(float x, float s_j, float scale, float r) {
+    return code8<FMT>(exact_value<MODE>(x, s_j, r), scale);
+}
+
 // |v| of one element, exactly (v as above).
 template <int MODE>
 __device__ __noinline__ float exact_abs(float x, float s_j, float r) {
@@ -823,12 +830,15 @@ struct RingPair {
     float* scale2 = nullptr;
 };
 
-template <int MODE, int R, int CPL, bool FULL, bool PAIR>
+template <int MODE, int R, int CPL, bool FULL, bool PAIR, int FMT>
 __global__ void __launch_bounds__(kRingThreads, 1)
 row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
                       int8_t* __restrict__ q, float* __restrict__ scale_out, float eps, float* __restrict__ r_out,
                       int ns, long long wait_limit, RingPair pr) {
     static_assert(!PAIR || MODE == kFold, "the pair launch folds its first tensor and smooths its second");
+    static_assert(!PAIR || FMT == kInt8, "the pair launch writes int8 codes");
+    static_assert(FMT == kInt8 || MODE != kNorm, "E4M3 codes for the fold and smoothing modes");
+    constexpr float kQmax = FMT == kE4M3 ? 448.0f : 127.0f;   // scale = amax / kQmax
     constexpr int G = kRingThreads / (32 * R);   // groups per CTA
     constexpr int NCP = 32 * R * CPL;            // chunks of a row padded to whole lanes
     constexpr uint32_t SLOT = NCP * 16u;         // bytes of one ring slot
@@ -1009,16 +1019,27 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             }
             const float a = group_max<R>(ex, red, grp, wig, lane, bank);
             bank ^= 1;
-            const float scale = a == 0.0f ? 1.0f : __fdiv_rn(a, 127.0f);
+            const float scale = a == 0.0f ? 1.0f : __fdiv_rn(a, kQmax);
 #pragma unroll 1
             for (int i = 0; i < CPL; ++i) {
                 const int c = gl + i * 32 * R;
                 if (c < nch) {
                     RawChunk<__nv_bfloat16> ch;
                     ch.a = *reinterpret_cast<const uint4*>(src + c * 16);
-                    *reinterpret_cast<uint2*>(rq + c * 8) =
-                        second ? exact_chunk_codes_in<__nv_bfloat16, kSmooth>(ch, s + c * 8, scale, rn, a == 0.0f)
-                               : exact_chunk_codes_in<__nv_bfloat16, MODE>(ch, s + c * 8, scale, rn, a == 0.0f);
+                    if (FMT == kInt8) {
+                        *reinterpret_cast<uint2*>(rq + c * 8) =
+                            second ? exact_chunk_codes_in<__nv_bfloat16, kSmooth>(ch, s + c * 8, scale, rn, a == 0.0f)
+                                   : exact_chunk_codes_in<__nv_bfloat16, MODE>(ch, s + c * 8, scale, rn, a == 0.0f);
+                    } else {
+                        // E4M3: an all-zero row keeps the signs of its zeros (scale 1)
+                        uint32_t b8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            b8[e] = exact_code_fmt<MODE, FMT>(ch.get(e), __ldg(s + c * 8 + e), scale, rn);
+                        *reinterpret_cast<uint2*>(rq + c * 8) =
+                            make_uint2(b8[0] | b8[1] << 8 | b8[2] << 16 | b8[3] << 24,
+                                       b8[4] | b8[5] << 8 | b8[6] << 16 | b8[7] << 24);
+                    }
                 }
             }
             if (gl == 0) so[row] = scale;
@@ -1051,14 +1072,14 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         }
 
         // ---- pass 2: codes
-        const float scale = __fdiv_rn(amax, 127.0f);
+        const float scale = __fdiv_rn(amax, kQmax);
         const float r = __frcp_rn(scale);
         const uint64_t r2 = f2_pack(r, r);
         uint32_t ntm = 0;
         uint2 codes[CPL];
+        if constexpr (FMT == kInt8) {
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            {
+            for (int i = 0; i < CPL; ++i) {
                 uint32_t t[8];
                 float dm = 0.0f;
 #pragma unroll
@@ -1075,6 +1096,30 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                 codes[i].x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
                 codes[i].y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
                 ntm |= (dm >= 0.5f - kTieGuard ? 1u : 0u) << i;   // (padding: d = 0)
+            }
+        } else {
+            // E4M3: q' = RN(v r) converted at q'(1 - 2^-18) and q'(1 + 2^-18);
+            // the conversion is monotone, and q* = RN(v / scale) lies within 6
+            // ulps of q' (within 2^-18 |q'|), so equal codes are q*'s code
+            const uint64_t lo2 = f2_pack(1.0f - 1.0f / 262144.0f, 1.0f - 1.0f / 262144.0f);
+            const uint64_t hi2 = f2_pack(1.0f + 1.0f / 262144.0f, 1.0f + 1.0f / 262144.0f);
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                uint32_t c16[4];
+                uint32_t diff = 0;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const uint64_t q2 = f2_mul(v2[i][p], r2);
+                    float l0, l1, h0, h1;
+                    f2_unpack(f2_mul(q2, lo2), l0, l1);
+                    f2_unpack(f2_mul(q2, hi2), h0, h1);
+                    const uint32_t cl = __nv_cvt_float2_to_fp8x2(make_float2(l0, l1), __NV_SATFINITE, __NV_E4M3);
+                    const uint32_t ch = __nv_cvt_float2_to_fp8x2(make_float2(h0, h1), __NV_SATFINITE, __NV_E4M3);
+                    diff |= cl ^ ch;
+                    c16[p] = cl;
+                }
+                codes[i] = make_uint2(c16[0] | c16[1] << 16, c16[2] | c16[3] << 16);
+                ntm |= (diff != 0u ? 1u : 0u) << i;   // (padding: zeros convert alike)
             }
         }
         // the stores apart from the arithmetic, which stays free of branches
@@ -1098,11 +1143,19 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             for (int e = 0; e < 8; ++e) {
                 const float x = bf16_elem(w, e);
                 const float vf = MODE == kNorm ? __fmul_rn(__fmul_rn(x, rn), mv[e]) : __fmul_rn(x, mv[e]);
-                const float tf = __fmaf_rn(vf, r, kMagic);
-                const float df = __fmaf_rn(vf, r, __fsub_rn(kMagic, tf));
-                if (fabsf(df) >= 0.5f - kTieGuard)
-                    rq[c * 8 + e] = (int8_t)(second ? exact_code<kSmooth>(x, __ldg(s + c * 8 + e), scale, rn)
-                                                    : exact_code<MODE>(x, __ldg(s + c * 8 + e), scale, rn));
+                bool redo;
+                if (FMT == kInt8) {
+                    const float tf = __fmaf_rn(vf, r, kMagic);
+                    const float df = __fmaf_rn(vf, r, __fsub_rn(kMagic, tf));
+                    redo = fabsf(df) >= 0.5f - kTieGuard;
+                } else {
+                    const float qf = __fmul_rn(vf, r);
+                    redo = __nv_cvt_float_to_fp8(__fmul_rn(qf, 1.0f - 1.0f / 262144.0f), __NV_SATFINITE, __NV_E4M3) !=
+                           __nv_cvt_float_to_fp8(__fmul_rn(qf, 1.0f + 1.0f / 262144.0f), __NV_SATFINITE, __NV_E4M3);
+                }
+                if (redo)
+                    rq[c * 8 + e] = (int8_t)(second ? exact_code_fmt<kSmooth, FMT>(x, __ldg(s + c * 8 + e), scale, rn)
+                                                    : exact_code_fmt<MODE, FMT>(x, __ldg(s + c * 8 + e), scale, rn));
             }
         }
     }
@@ -1205,13 +1258,13 @@ size_t ring_smem_bytes(int R, int CPL, int ns, bool pair) {
     return ncp * (pair ? 64 : 32) + G * (size_t)ns * (ncp * 16 + 8) + G * 2 * (size_t)R * (4 + 8);
 }
 
-template <int MODE, int R, int CPL, bool FULL, bool PAIR>
+template <int MODE, int R, int CPL, bool FULL, bool PAIR, int FMT>
 sq_status launch_row_quant_ring_inst(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
                                      float* scale, cudaStream_t st, float eps, float* r_out, int ns,
                                      const RingPair& pr) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
-    auto kern = row_quant_ring_kernel<MODE, R, CPL, FULL, PAIR>;
+    auto kern = row_quant_ring_kernel<MODE, R, CPL, FULL, PAIR, FMT>;
     if (!attr_done[di.device & 63]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row_quant_ring_kernel)");
@@ -1225,16 +1278,23 @@ sq_status launch_row_quant_ring_inst(const void* in, int64_t rows, int64_t K, co
                       wait_limit_cycles(), pr);
 }
 
-template <int MODE, int R, bool PAIR>
+template <int MODE, int R, bool PAIR, int FMT>
 sq_status launch_row_quant_ring_r(int cpl, const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
                                   float* scale, cudaStream_t st, float eps, float* r_out, int ns,
                                   const RingPair& pr) {
-    // rows that fill every lane (K = 256 R CPL) drop the stores' bounds checks
+    // rows that fill every lane (K = 256 R CPL) drop the stores' bounds checks;
+    // E4M3 codes are instantiated for such rows only (the caller checks)
     const bool full = K / 8 == (int64_t)32 * R * cpl;
-#define SQ_RING_CPL(C)                                                                                          \
-    return full ? launch_row_quant_ring_inst<MODE, R, C, true, PAIR>(in, rows, K, s, q, scale, st, eps, r_out, ns, \
-                                                                     pr)                                          \
-                : launch_row_quant_ring_inst<MODE, R, C, false, PAIR>(in, rows, K, s, q, scale, st, eps, r_out, ns, pr)
+#define SQ_RING_CPL(C)                                                                                            \
+    if constexpr (FMT == kInt8) {                                                                                 \
+        return full ? launch_row_quant_ring_inst<MODE, R, C, true, PAIR, FMT>(in, rows, K, s, q, scale, st, eps,  \
+                                                                              r_out, ns, pr)                      \
+                    : launch_row_quant_ring_inst<MODE, R, C, false, PAIR, FMT>(in, rows, K, s, q, scale, st, eps, \
+                                                                               r_out, ns, pr);                    \
+    } else {                                                                                                      \
+        return launch_row_quant_ring_inst<MODE, R, C, true, PAIR, FMT>(in, rows, K, s, q, scale, st, eps, r_out,  \
+                                                                       ns, pr);                                   \
+    }
     if constexpr (R == 2) {
         if (cpl == 10) { SQ_RING_CPL(10); }
     }
@@ -1255,7 +1315,7 @@ sq_status launch_row_quant_ring_r(int cpl, const void* in, int64_t rows, int64_t
 // faster than three or four). Returns false when K is outside that range or
 // the padded row, its multipliers and two slots exceed the shared memory of a
 // CTA (K above 28672).
-template <int MODE, bool PAIR = false>
+template <int MODE, bool PAIR = false, int FMT = kInt8>
 bool launch_row_quant_ring(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q, float* scale,
                            cudaStream_t st, float eps, float* r_out, sq_status& result,
                            const RingPair& pr = RingPair{}) {
@@ -1273,12 +1333,15 @@ bool launch_row_quant_ring(const void* in, int64_t rows, int64_t K, const float*
     }
     const int ns = 2;
     if (ring_smem_bytes(R, cpl, ns, PAIR) > kRingSmemMax) return false;
+    if (FMT != kInt8 && nchunks != (int64_t)32 * R * cpl) return false;
+#define SQ_RING_R(RR) launch_row_quant_ring_r<MODE, RR, PAIR, FMT>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr)
     switch (R) {
-        case 2: result = launch_row_quant_ring_r<MODE, 2, PAIR>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr); break;
-        case 4: result = launch_row_quant_ring_r<MODE, 4, PAIR>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr); break;
-        case 8: result = launch_row_quant_ring_r<MODE, 8, PAIR>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr); break;
-        default: result = launch_row_quant_ring_r<MODE, 16, PAIR>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr); break;
+        case 2: result = SQ_RING_R(2); break;
+        case 4: result = SQ_RING_R(4); break;
+        case 8: result = SQ_RING_R(8); break;
+        default: result = SQ_RING_R(16); break;
     }
+#undef SQ_RING_R
     return true;
 }
 
@@ -1475,6 +1538,14 @@ static sq_status row_quant_e4m3_common(int mode, const void* in, sq_dtype dt, in
     if (!s || !q || !scale) { set_error("NULL pointer"); return SQ_ERR_INVALID_ARG; }
     if (!aligned16(s) || !aligned16(q)) { set_error("s and codes must be 16-byte aligned"); return SQ_ERR_UNSUPPORTED; }
     int8_t* qq = reinterpret_cast<int8_t*>(q);
+    if (dt == SQ_BF16) {
+        // rows that fill the streamed kernel's lanes exactly: the fast E4M3 pass
+        sq_status res = SQ_OK;
+        if (mode == kFold ? launch_row_quant_ring<kFold, false, kE4M3>(in, rows, K, s, qq, scale, st, 0.0f, nullptr, res)
+                          : launch_row_quant_ring<kSmooth, false, kE4M3>(in, rows, K, s, qq, scale, st, 0.0f, nullptr,
+                                                                         res))
+            return res;
+    }
     if (mode == kFold)
         return dt == SQ_F32 ? launch_row_quant_exact<float, kFold, kE4M3>(in, rows, K, s, qq, scale, st)
                             : launch_row_quant_exact<__nv_bfloat16, kFold, kE4M3>(in, rows, K, s, qq, scale, st);
