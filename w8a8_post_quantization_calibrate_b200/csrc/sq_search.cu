@@ -223,8 +223,7 @@ sq_status alpha_search_impl(const void* x, const void* w, sq_dtype dt, int64_t T
     if (blocks > kErrMaxBlocks) blocks = kErrMaxBlocks;
     for (int64_t a = 0; a < n_alpha; ++a) {
         if ((r = smooth_factors_impl(xmax, wmax, K, alphas[a], eps, s, st)) != SQ_OK) return r;
-        if ((r = fold_quant_weights_impl(w, dt, N, K, s, wq, wsc, st)) != SQ_OK) return r;
-        if ((r = smooth_quant_act_impl(x, dt, T, K, s, xq, xs, st)) != SQ_OK) return r;
+        if ((r = fold_smooth_quant_pair_impl(w, N, x, T, dt, K, s, wq, wsc, xq, xs, st)) != SQ_OK) return r;
         if ((r = gemm_dispatch(xq, xs, wq, wsc, T, N, K, yq, SQ_F32, base + L.gemm_ws, L.gemm_ws_bytes, st)) != SQ_OK)
             return r;
         err_partial_kernel<<<blocks, kErrThreads, 0, st>>>(yq, yref, nel, part);
