@@ -168,7 +168,9 @@ sq_status tensor_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_t c
     if (rows == 0 || cols == 0) return SQ_OK;
     dim3 grid;
     int64_t per = 0;
-    if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
+    const int per_sm = dt == SQ_F32 ? column_blocks_per_sm<col_absmax_kernel<float, true>>()
+                                    : column_blocks_per_sm<col_absmax_kernel<__nv_bfloat16, true>>();
+    if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per, per_sm)) != SQ_OK) return r;
     if (dt == SQ_F32)
         return launch_pdl("col_absmax_kernel<tensor>", col_absmax_kernel<float, true>, grid, dim3(kAbsmaxThreads), 0,
                           st, 1, static_cast<const uint8_t*>(x), rows, cols, per, amax, s, AbsmaxPair{});
@@ -187,7 +189,9 @@ sq_status quant_act_per_tensor_impl(const void* x, sq_dtype dt, int64_t T, int64
     if (!aligned16(xq)) { set_error("codes must be 16-byte aligned"); return SQ_ERR_UNSUPPORTED; }
     dim3 grid;
     int64_t per = 0;
-    if ((r = absmax_grid(T, K, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
+    const int per_sm = dt == SQ_F32 ? column_blocks_per_sm<per_tensor_quant_kernel<float>>()
+                                    : column_blocks_per_sm<per_tensor_quant_kernel<__nv_bfloat16>>();
+    if ((r = absmax_grid(T, K, dt == SQ_F32 ? 4 : 2, grid, per, per_sm)) != SQ_OK) return r;
     if (dt == SQ_F32)
         return launch_pdl("per_tensor_quant_kernel", per_tensor_quant_kernel<float>, grid, dim3(kAbsmaxThreads), 0, st,
                           1, static_cast<const uint8_t*>(x), T, K, per, s, amax, xq, x_scale);

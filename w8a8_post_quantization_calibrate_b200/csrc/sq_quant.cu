@@ -1407,14 +1407,27 @@ sq_status check_matrix(const void* p, int64_t rows, int64_t cols, const char* na
 
 }  // namespace
 
-// About one wave of 256-thread blocks (8 per SM); every block covers a
-// multiple of the 64 rows it reads per iteration. Returns the grid and the rows
-// per block.
-sq_status absmax_grid(int64_t rows, int64_t cols, int es, dim3& grid, int64_t& per) {
+// Resident 256-thread blocks per SM of a column kernel (its registers and
+// static shared memory decide; looked up once per kernel).
+template <auto KERN>
+int column_blocks_per_sm() {
+    static int cached = 0;
+    if (cached == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, KERN, kAbsmaxThreads, 0) != cudaSuccess || n < 1) n = 1;
+        cached = n;
+    }
+    return cached;
+}
+
+// One full wave of 256-thread blocks (per_sm resident per SM); every block
+// covers a multiple of the 64 rows it reads per iteration. Returns the grid
+// and the rows per block.
+sq_status absmax_grid(int64_t rows, int64_t cols, int es, dim3& grid, int64_t& per, int per_sm) {
     const int64_t tile = 32 * (16 / es);
     const int64_t ct = (cols + tile - 1) / tile;
     const int64_t step_rows = 8 * kAbsmaxRowsInFlight;
-    const int64_t target = (int64_t)device_info().sm_count * 8;
+    const int64_t target = (int64_t)device_info().sm_count * per_sm;
     int64_t rc = target / ct;
     if (rc < 1) rc = 1;
     per = (rows + rc - 1) / rc;
@@ -1440,7 +1453,9 @@ sq_status calibrate_absmax_impl(const void* x, sq_dtype dt, int64_t rows, int64_
     if (rows == 0 || cols == 0) return SQ_OK;
     dim3 grid;
     int64_t per = 0;
-    if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per)) != SQ_OK) return r;
+    const int per_sm = dt == SQ_F32 ? column_blocks_per_sm<col_absmax_kernel<float, false>>()
+                                    : column_blocks_per_sm<col_absmax_kernel<__nv_bfloat16, false>>();
+    if ((r = absmax_grid(rows, cols, dt == SQ_F32 ? 4 : 2, grid, per, per_sm)) != SQ_OK) return r;
     if (dt == SQ_F32)
         return launch_pdl("col_absmax_kernel", col_absmax_kernel<float, false>, grid, dim3(kAbsmaxThreads), 0, st, 1,
                           static_cast<const uint8_t*>(x), rows, cols, per, absmax, (const float*)nullptr,
@@ -1466,7 +1481,9 @@ sq_status calibrate_absmax_pair_impl(const void* x, int64_t T, const void* w, in
     const int64_t ct = (K + tile - 1) / tile;
     if (ct > 2147483647LL) { set_error("cols too large"); return SQ_ERR_UNSUPPORTED; }
     const int64_t step_rows = 8 * kAbsmaxRowsInFlight;
-    const int64_t target = (int64_t)device_info().sm_count * 8;
+    const int per_sm = dt == SQ_F32 ? column_blocks_per_sm<col_absmax_kernel<float, false>>()
+                                    : column_blocks_per_sm<col_absmax_kernel<__nv_bfloat16, false>>();
+    const int64_t target = (int64_t)device_info().sm_count * per_sm;
     auto chunks = [&](int64_t rows, int64_t share, int64_t& per) {
         int64_t rc = share / ct;
         if (rc < 1) rc = 1;
