@@ -362,6 +362,13 @@ sq_status sq_fold_quant_weights_e4m3(const void* w, sq_dtype dt, int64_t N, int6
                                      uint8_t* wq, float* w_scale, sq_stream_t stream);
 sq_status sq_smooth_quant_act_e4m3(const void* x, sq_dtype dt, int64_t T, int64_t K, const float* s,
                                    uint8_t* xq, float* x_scale, sq_stream_t stream);
+/* sq_fold_smooth_quant_pair_e4m3: sq_fold_quant_weights_e4m3 on w [N x K] and
+ *   sq_smooth_quant_act_e4m3 on x [T x K] with the same s, in one launch where
+ *   the library's streamed row kernel takes both (bf16 rows that fill its
+ *   lanes), else the two calls; same results, bit for bit. */
+sq_status sq_fold_smooth_quant_pair_e4m3(const void* w, int64_t N, const void* x, int64_t T, sq_dtype dt, int64_t K,
+                                         const float* s, uint8_t* wq, float* w_scale, uint8_t* xq, float* x_scale,
+                                         sq_stream_t stream);
 sq_status sq_w8a8_gemm_e4m3(const uint8_t* xq, const float* x_scale, const uint8_t* wq,
                             const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
                             sq_dtype out_dt, sq_stream_t stream);

@@ -65,6 +65,12 @@ def test_host_argument_checks(sq):
                          dummy, st) == sq.SQ_ERR_INVALID_ARG
     assert sq.raw_status("sq_fold_smooth_quant_pair", dummy, 0, dummy, 0, sq.SQ_BF16, 16, dummy, dummy, dummy, dummy,
                          dummy, st) == sq.SQ_OK   # no-op
+    assert sq.raw_status("sq_fold_smooth_quant_pair_e4m3", dummy, 8, dummy, 4, sq.SQ_I32, 16, dummy, dummy, dummy,
+                         dummy, dummy, st) == sq.SQ_ERR_UNSUPPORTED
+    assert sq.raw_status("sq_fold_smooth_quant_pair_e4m3", dummy, 8, dummy, 4, sq.SQ_BF16, 24, dummy, dummy, dummy,
+                         dummy, dummy, st) == sq.SQ_ERR_UNSUPPORTED
+    assert sq.raw_status("sq_fold_smooth_quant_pair_e4m3", dummy, 8, dummy, 4, sq.SQ_BF16, 16, None, dummy, dummy,
+                         dummy, dummy, st) == sq.SQ_ERR_INVALID_ARG
     assert sq.raw_status("sq_smooth_quant_act", dummy, sq.SQ_BF16, 8, 24, dummy, dummy, dummy, st) \
         == sq.SQ_ERR_UNSUPPORTED
     assert sq.raw_status("sq_smooth_quant_act", dummy, sq.SQ_BF16, 8, 16, None, dummy, dummy, st) \

@@ -218,3 +218,32 @@ def test_e4m3_stream_kernel_rows(K):
     oq, osc = oracle.fold_quant_weights_e4m3(hx, s)
     assert_equal(host(q), oq, "E4M3 fold codes")
     assert_bitexact_f32(host(sc), osc, "E4M3 fold scales")
+
+
+@pytest.mark.parametrize("N,T,K", [(300, 37, 4096), (70, 90, 5120), (9, 5, 28672), (20, 12, 11008), (40, 3, 1040)])
+def test_e4m3_pair_launch_equals_the_two_calls(N, T, K):
+    """FP8 codes of the weights and the activations in one launch (the
+    streamed kernel where the rows fill its lanes; K = 28672, 11008 and 1040
+    take the two calls): the same bytes and scales as the two calls and the
+    oracle."""
+    g = torch.Generator().manual_seed(N + 2 * T + K)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    x = outlier_x(T, K, torch.bfloat16, seed=N + K)
+    if T > 2:
+        x[1] = 0.0
+        x[2] *= 1e-33
+    s = s_for(K, K + 9)
+    sd, wd, xd = dev(torch.from_numpy(s)), dev(w), dev(x)
+    wq, wsc, xq, xsc = sq.sq_fold_smooth_quant_pair_e4m3(wd, xd, sd)
+    wq1, wsc1 = sq.sq_fold_quant_weights_e4m3(wd, sd)
+    xq1, xsc1 = sq.sq_smooth_quant_act_e4m3(xd, sd)
+    assert_equal(host(wq), host(wq1), "pair vs separate: wq")
+    assert_equal(host(xq), host(xq1), "pair vs separate: xq")
+    assert_bitexact_f32(host(wsc), host(wsc1), "pair vs separate: w_scale")
+    assert_bitexact_f32(host(xsc), host(xsc1), "pair vs separate: x_scale")
+    oq, osc = oracle.fold_quant_weights_e4m3(synth.host_array(w), s)
+    assert_equal(host(wq), oq, "pair wq vs oracle")
+    assert_bitexact_f32(host(wsc), osc, "pair w_scale vs oracle")
+    oq, osc = oracle.smooth_quant_act_e4m3(synth.host_array(x), s)
+    assert_equal(host(xq), oq, "pair xq vs oracle")
+    assert_bitexact_f32(host(xsc), osc, "pair x_scale vs oracle")

@@ -836,7 +836,6 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                       int8_t* __restrict__ q, float* __restrict__ scale_out, float eps, float* __restrict__ r_out,
                       int ns, long long wait_limit, RingPair pr) {
     static_assert(!PAIR || MODE == kFold, "the pair launch folds its first tensor and smooths its second");
-    static_assert(!PAIR || FMT == kInt8, "the pair launch writes int8 codes");
     static_assert(FMT == kInt8 || MODE != kNorm, "E4M3 codes for the fold and smoothing modes");
     constexpr float kQmax = FMT == kE4M3 ? 448.0f : 127.0f;   // scale = amax / kQmax
     constexpr int G = kRingThreads / (32 * R);   // groups per CTA
@@ -1035,7 +1034,8 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                         uint32_t b8[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            b8[e] = exact_code_fmt<MODE, FMT>(ch.get(e), __ldg(s + c * 8 + e), scale, rn);
+                            b8[e] = second ? exact_code_fmt<kSmooth, FMT>(ch.get(e), __ldg(s + c * 8 + e), scale, rn)
+                                           : exact_code_fmt<MODE, FMT>(ch.get(e), __ldg(s + c * 8 + e), scale, rn);
                         *reinterpret_cast<uint2*>(rq + c * 8) =
                             make_uint2(b8[0] | b8[1] << 8 | b8[2] << 16 | b8[3] << 24,
                                        b8[4] | b8[5] << 8 | b8[6] << 16 | b8[7] << 24);
@@ -1545,8 +1545,8 @@ static sq_status row_quant_common(int mode, const void* in, sq_dtype dt, int64_t
 
 // FP8 E4M3 codes: the same fold / smoothing, per-row scale amax / 448, every
 // quotient an IEEE division (the exact kernel).
-static sq_status row_quant_e4m3_common(int mode, const void* in, sq_dtype dt, int64_t rows, int64_t K,
-                                       const float* s, uint8_t* q, float* scale, cudaStream_t st) {
+sq_status row_quant_e4m3_common(int mode, const void* in, sq_dtype dt, int64_t rows, int64_t K,
+                                const float* s, uint8_t* q, float* scale, cudaStream_t st) {
     sq_status r;
     if ((r = check_input_dtype(dt)) != SQ_OK) return r;
     if ((r = check_matrix(in, rows, K, "input")) != SQ_OK) return r;
@@ -1611,6 +1611,36 @@ sq_status fold_smooth_quant_pair_impl(const void* w, int64_t N, const void* x, i
     return smooth_quant_act_impl(x, dt, T, K, s, xq, x_scale, st);
 }
 
+// The same pair with FP8 E4M3 codes: one launch where the streamed kernel's
+// E4M3 pass takes both (bf16 rows that fill its lanes, two multiplier tables
+// beside the ring); else the two E4M3 calls.
+sq_status fold_smooth_quant_pair_e4m3_impl(const void* w, int64_t N, const void* x, int64_t T, sq_dtype dt,
+                                           int64_t K, const float* s, uint8_t* wq, float* w_scale, uint8_t* xq,
+                                           float* x_scale, cudaStream_t st) {
+    sq_status r;
+    if ((r = check_input_dtype(dt)) != SQ_OK) return r;
+    if ((r = check_matrix(w, N, K, "w")) != SQ_OK) return r;
+    if ((r = check_matrix(x, T, K, "x")) != SQ_OK) return r;
+    if (dt == SQ_BF16 && N > 0 && T > 0 && K > 0) {
+        if (!s || !wq || !w_scale || !xq || !x_scale) { set_error("NULL pointer"); return SQ_ERR_INVALID_ARG; }
+        if (!aligned16(s) || !aligned16(wq) || !aligned16(xq)) {
+            set_error("s and codes must be 16-byte aligned");
+            return SQ_ERR_UNSUPPORTED;
+        }
+        RingPair pr;
+        pr.in2 = static_cast<const __nv_bfloat16*>(x);
+        pr.rows2 = T;
+        pr.q2 = reinterpret_cast<int8_t*>(xq);
+        pr.scale2 = x_scale;
+        sq_status res = SQ_OK;
+        if (launch_row_quant_ring<kFold, true, kE4M3>(w, N, K, s, reinterpret_cast<int8_t*>(wq), w_scale, st, 0.0f,
+                                                      nullptr, res, pr))
+            return res;
+    }
+    if ((r = row_quant_e4m3_common(kFold, w, dt, N, K, s, wq, w_scale, st)) != SQ_OK) return r;
+    return row_quant_e4m3_common(kSmooth, x, dt, T, K, s, xq, x_scale, st);
+}
+
 }  // namespace sq
 
 extern "C" {
@@ -1623,6 +1653,13 @@ sq_status sq_fold_quant_weights_e4m3(const void* w, sq_dtype dt, int64_t N, int6
 sq_status sq_smooth_quant_act_e4m3(const void* x, sq_dtype dt, int64_t T, int64_t K, const float* s, uint8_t* xq,
                                    float* x_scale, sq_stream_t stream) {
     return sq::row_quant_e4m3_common(sq::kSmooth, x, dt, T, K, s, xq, x_scale, (cudaStream_t)stream);
+}
+
+sq_status sq_fold_smooth_quant_pair_e4m3(const void* w, int64_t N, const void* x, int64_t T, sq_dtype dt, int64_t K,
+                                         const float* s, uint8_t* wq, float* w_scale, uint8_t* xq, float* x_scale,
+                                         sq_stream_t stream) {
+    return sq::fold_smooth_quant_pair_e4m3_impl(w, N, x, T, dt, K, s, wq, w_scale, xq, x_scale,
+                                                (cudaStream_t)stream);
 }
 
 

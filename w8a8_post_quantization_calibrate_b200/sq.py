@@ -45,6 +45,7 @@ _SIGS = {
     "sq_smooth_quant_act": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_calibrate_absmax_pair": ([_vp, _i64, _vp, _i64, _int, _i64, _vp, _vp, _vp], _int),
     "sq_fold_smooth_quant_pair": ([_vp, _i64, _vp, _i64, _int, _i64, _vp, _vp, _vp, _vp, _vp, _vp], _int),
+    "sq_fold_smooth_quant_pair_e4m3": ([_vp, _i64, _vp, _i64, _int, _i64, _vp, _vp, _vp, _vp, _vp, _vp], _int),
     "sq_fold_quant_weights_e4m3": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_smooth_quant_act_e4m3": ([_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp], _int),
     "sq_w8a8_gemm_e4m3": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp], _int),
@@ -197,6 +198,29 @@ def sq_fold_smooth_quant_pair(w: torch.Tensor, x: torch.Tensor, s: torch.Tensor,
     _check(_lib.sq_fold_smooth_quant_pair(_dev(w, "w"), N, _dev(x, "x"), T, _dt(w), K, _dev(s, "s"), _dev(wq, "wq"),
                                           _dev(w_scale, "w_scale"), _dev(xq, "xq"), _dev(x_scale, "x_scale"),
                                           _stream(stream)), "sq_fold_smooth_quant_pair")
+    return wq, w_scale, xq, x_scale
+
+
+def sq_fold_smooth_quant_pair_e4m3(w: torch.Tensor, x: torch.Tensor, s: torch.Tensor, wq=None, w_scale=None,
+                                   xq=None, x_scale=None, stream=None):
+    """FP8 E4M3 codes of w (folded) and x (smoothed) in one launch where
+    possible -> (wq uint8, w_scale, xq uint8, x_scale)."""
+    N, K = w.shape
+    T = x.shape[0]
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must have the same dtype")
+    if wq is None:
+        wq = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=w.device)
+    if xq is None:
+        xq = torch.empty((T, K), dtype=torch.uint8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(_lib.sq_fold_smooth_quant_pair_e4m3(_dev(w, "w"), N, _dev(x, "x"), T, _dt(w), K, _dev(s, "s"),
+                                               _dev(wq, "wq"), _dev(w_scale, "w_scale"), _dev(xq, "xq"),
+                                               _dev(x_scale, "x_scale"), _stream(stream)),
+           "sq_fold_smooth_quant_pair_e4m3")
     return wq, w_scale, xq, x_scale
 
 
