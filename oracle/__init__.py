@@ -46,6 +46,7 @@ MUTATIONS = {
     "split_max_all": 16,
     "split_drop_outliers": 17,
     "e4m3_truncate": 18,
+    "pow_exponent": 19,
 }
 
 _lock = threading.Lock()

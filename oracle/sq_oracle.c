@@ -68,7 +68,8 @@ enum {
     MUT_NORM_MEAN_ABS = 15,    /* RMSNorm from the mean |x| instead of the mean square */
     MUT_SPLIT_MAX_ALL = 16,    /* bulk scale taken over the outlier channels too */
     MUT_SPLIT_DROP_OUTLIERS = 17, /* decomposition forgets the floating-point term */
-    MUT_E4M3_TRUNCATE = 18     /* FP8 E4M3 conversion truncates instead of rounding */
+    MUT_E4M3_TRUNCATE = 18,    /* FP8 E4M3 conversion truncates instead of rounding */
+    MUT_POW_EXPONENT = 19      /* generic alpha: pow(v, 1 - a) instead of pow(v, a) */
 };
 static int g_mutation = MUT_NONE;
 
@@ -209,6 +210,7 @@ static double pow_alpha(double v, double a)
     if (a == 0.5) return sqrt(v);
     if (a == 0.25) return sqrt(sqrt(v));
     if (a == 0.75) return sqrt(v) * sqrt(sqrt(v));
+    if (g_mutation == MUT_POW_EXPONENT) return pow(v, 1.0 - a);
     return pow(v, a);
 }
 

@@ -178,6 +178,46 @@ def pin_alpha_closed_forms():
         assert abs(float(sh[j]) - ref) <= ulp32(ref), (j, sh[j], ref)
 
 
+def _pow_dec(v: float, a: Fraction):
+    """v**a for an fp32 value v and a rational exponent, to 50 significant
+    digits (the decimal module's ln and exp are correctly rounded)."""
+    import decimal
+    ctx = decimal.Context(prec=50)
+    dv = ctx.create_decimal_from_float(float(v))
+    da = ctx.divide(decimal.Decimal(a.numerator), decimal.Decimal(a.denominator))
+    return ctx.exp(ctx.multiply(da, ctx.ln(dv)))
+
+
+def pin_alpha_generic_pow():
+    """alpha outside {0, 1/4, 1/2, 3/4, 1} goes through the general power.
+    (1) Dyadic alphas on powers of two give exact powers of two:
+    xmax = 2^(8k), wmax = 2^(-8m), alpha = p/8 -> s = 2^(k p + m (8 - p)).
+    (2) The alphas the tests use (0.3, 0.4, 0.6, 0.85 as fp32) on random
+    maxima: s within 1 fp32 ulp of xmax^alpha / wmax^(1-alpha) evaluated to
+    50 digits, with alpha taken exactly as the fp32 value the call receives."""
+    for p in (1, 3, 5, 7):
+        a = np.float32(p / 8)
+        ks = [-3, -1, 0, 1, 2, 4]
+        ms = [-2, 0, 1, 3, 5, 7]
+        xmax = np.array([2.0 ** (8 * k) for k in ks], np.float32)
+        wmax = np.array([2.0 ** (-8 * m) for m in ms], np.float32)
+        s = oracle.smooth_factors(xmax, wmax, float(a), 0.0)
+        for j, (k, m) in enumerate(zip(ks, ms)):
+            want = np.float32(2.0 ** (k * p + m * (8 - p)))
+            assert _bits(s[j]) == _bits(want), (p, k, m, s[j], want)
+    rng = np.random.default_rng(19)
+    xmax = rng.uniform(0.05, 90.0, 48).astype(np.float32)
+    wmax = rng.uniform(0.002, 0.6, 48).astype(np.float32)
+    for av in (0.3, 0.4, 0.6, 0.85):
+        a32 = np.float32(av)
+        a = Fraction(float(a32))
+        s = oracle.smooth_factors(xmax, wmax, float(a32), 1e-8)
+        for j in range(48):
+            exact = _pow_dec(xmax[j], a) / _pow_dec(wmax[j], 1 - a)
+            ref = float(exact)
+            assert abs(float(s[j]) - ref) <= ulp32(ref), (av, j, float(s[j]), ref)
+
+
 def _outlier_xw(T=96, K=256, N=80, seed=5):
     rng = np.random.default_rng(seed)
     X = rng.standard_normal((T, K))
@@ -486,6 +526,7 @@ FAST_PINS = [
     pin_near_ties_exact,
     pin_log2k_intervals,
     pin_alpha_closed_forms,
+    pin_alpha_generic_pow,
     pin_migration_invariants,
     pin_smoothing_identity,
     pin_calibration_absmax,
