@@ -1,13 +1,21 @@
 #!/usr/bin/env python3
 """Benchmark of the SmoothQuant W8A8 smoothed linear layer on B200.
 
-One step = one pass of the whole path over one batch of the 7B-like QKV
-projection prefill workload (X bf16 [4096 x 4096] with 0.1% outlier channels,
-W bf16 [12288 x 4096], alpha 0.5, bf16 output):
-  a1 calibrate X and W -> a2 smoothing factors -> a3 fold + quantize W ->
-  a4 smooth + quantize X -> a5 int8 GEMM with dequant epilogue,
-each a call into libsq's C ABI on one CUDA stream. L2 is flushed between
-steps; every kernel is bracketed by CUDA events on that stream.
+The measured workload is the 70B-like down projection prefill: X bf16
+[8192 x 28672] with 0.05% outlier channels, W bf16 [8192 x 28672], bf16 output.
+One step = one pass of the whole path over one batch, each stage a call into
+libsq's C ABI on one CUDA stream:
+  a1 calibrate: the activation maxima over 16 seeded calibration batches of
+     2048 tokens (resident in HBM, read in one launch: the running maximum
+     over batches equals the maximum over their concatenation) and the
+     weight maxima, in one launch;
+  a2 smoothing factors at alpha = 0.5;
+  a3 fold + quantize W;  a4 smooth + quantize X;
+  a5 int8 GEMM with the dequantizing epilogue.
+The alpha sweep {0.25, 0.5, 0.75} (a2..a5 per alpha, after the same
+calibration) is timed and reported per alpha in the same line. L2 is flushed
+between steps. Other configurations (--workload) and activation variants
+(--variant) serve profiling.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -34,13 +42,15 @@ sys.path.insert(0, ROOT)
 from w8a8_post_quantization_calibrate_b200 import synth  # noqa: E402
 
 METRIC = "W8A8 smoothed-linear int8 TOPS & act-quant GB/s at 1 B200; % of roofline"
-WORKLOAD = "qkv_prefill_7b"
+WORKLOAD = "down_prefill_70b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # datasheet figures, reported beside the measured denominators for context only
 SPEC_HBM_GBS = 8000.0
 SPEC_INT8_TOPS = 4500.0
 INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOP/s bf16)
 L2_FLUSH_BYTES = 256 << 20
+PROBE_ITERS = 4096      # one probe launch: about the length of the 70B GEMM
+PROBE_LAUNCHES = 20
 
 
 # ------------------------------------------------------------------ helpers
@@ -66,9 +76,10 @@ def gemm_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def load_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu summary, or None when
-    absent or taken on a different version of the kernel source."""
+def load_traffic(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary for this
+    workload, or None when absent or taken on another version of the kernel
+    source."""
     p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if not os.path.exists(p):
         return None
@@ -76,7 +87,8 @@ def load_traffic():
         d = json.load(f)
     if d.get("source_sha256_16") != gemm_source_hash():
         return None
-    return d.get("dram_bytes_per_launch")
+    per = d.get("per_workload", {}).get(workload)
+    return None if per is None else per.get("dram_bytes_per_launch")
 
 
 def dist_env():
@@ -105,19 +117,32 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 class ClockSampler:
     """Samples SM clock, power and clock-event reasons through NVML while the
-    timed region runs (reads only; changes no setting)."""
+    timed region runs (reads only; changes no setting). mark() labels the
+    samples taken from then on."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
                0x10: "sync_boost", 0x1: "gpu_idle"}
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
         self.err = None
+        self.label = "setup"
         self._stop = threading.Event()
         try:
             import pynvml
@@ -130,6 +155,9 @@ class ClockSampler:
             self.err = repr(e)
         self._t = threading.Thread(target=self._run, daemon=True)
 
+    def mark(self, label: str):
+        self.label = label
+
     def _run(self):
         while not self._stop.is_set():
             try:
@@ -137,7 +165,7 @@ class ClockSampler:
                 util = self.nvml.nvmlDeviceGetUtilizationRates(self.h).gpu
                 reasons = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
                 pw = self.nvml.nvmlDeviceGetPowerUsage(self.h) / 1000.0
-                self.samples.append((sm, util, reasons, pw))
+                self.samples.append((sm, util, reasons, pw, self.label))
             except Exception as e:  # pragma: no cover
                 self.err = repr(e)
             self._stop.wait(self.period)
@@ -152,60 +180,114 @@ class ClockSampler:
         if self.nvml is not None:
             self._t.join()
 
-    def summary(self):
-        if not self.samples:
+    def summary(self, labels=None):
+        pick = [s for s in self.samples if labels is None or s[4] in labels]
+        if not pick:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
                     "note": self.err or "no samples"}
-        loaded = [s for s in self.samples if s[1] > 0] or self.samples
+        loaded = [s for s in pick if s[1] > 0] or pick
         seen = 0
         for s in loaded:
             seen |= s[2]
         reasons = [name for bit, name in self.REASONS.items() if seen & bit and name != "gpu_idle"]
         return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(loaded),
+                "sm_mhz_min": min(s[0] for s in loaded), "reasons": sorted(reasons), "samples": len(loaded),
                 "power_w_max": round(max(s[3] for s in loaded), 1)}
 
 
+def median(v):
+    return statistics.median(v) if v else float("nan")
+
+
 # ------------------------------------------------------------------ the CPU oracle
-def oracle_sample(x: torch.Tensor, w: torch.Tensor, alpha: float, seconds: float,
-                  tokens: int = 64, rows: int = 256):
-    """The oracle, as it stands, on a bounded sample of the workload: the whole
-    path on a slice of `tokens` tokens x `rows` output channels (full K),
-    repeated until `seconds` have passed. Returns (TOPS, threads, description,
-    seconds per slice)."""
+def _timed(fn, *a):
+    t0 = time.perf_counter()
+    out = fn(*a)
+    return out, time.perf_counter() - t0
+
+
+def oracle_stages(x_cpu, w_cpu, alpha, xcal_cpu=None, gemm_rows=256):
+    """The oracle, as it stands, per stage on the workload's full tensors (a1
+    over the calibration tensor and W, a2, a3 over all of W, a4 over all of X)
+    and a5 on the first `gemm_rows` tokens, plus one-thread figures of a3, a4
+    and a5 on bounded slices. Returns (stages dict, whole-path TOPS estimate,
+    description)."""
+    import oracle
+    hx = synth.host_array(x_cpu)
+    hw = synth.host_array(w_cpu)
+    hc = hx if xcal_cpu is None else synth.host_array(xcal_cpu)
+    M, K = hx.shape
+    N = hw.shape[0]
+    ies = x_cpu.element_size()
+    threads = oracle.num_threads()
+    st = {}
+    xmax, t1x = _timed(oracle.col_absmax, hc)
+    wmax, t1w = _timed(oracle.col_absmax, hw)
+    st["a1_calibrate_xw"] = {"s": t1x + t1w, "gbs": (hc.size + hw.size) * ies / (t1x + t1w) / 1e9}
+    s, t2 = _timed(oracle.smooth_factors, xmax, wmax, alpha)
+    st["a2_smooth_factors"] = {"s": t2}
+    (wq, wsc), t3 = _timed(oracle.fold_quant_weights, hw, s)
+    st["a3_fold_quant_w"] = {"s": t3, "gbs": (hw.size * (ies + 1) + 4 * (N + K)) / t3 / 1e9}
+    (xq, xsc), t4 = _timed(oracle.smooth_quant_act, hx, s)
+    st["a4_smooth_quant_x"] = {"s": t4, "gbs": (hx.size * (ies + 1) + 4 * (M + K)) / t4 / 1e9}
+    rows = min(gemm_rows, M)
+    _, t5 = _timed(oracle.gemm_i8, np.ascontiguousarray(xq[:rows]), wq)
+    t5_full = t5 * M / rows
+    st["a5_w8a8_gemm"] = {"s_slice": t5, "rows": rows, "tops_slice": 2.0 * rows * N * K / t5 / 1e12,
+                          "s_extrapolated": t5_full}
+    # one thread, bounded slices
+    oracle.set_num_threads(1)
+    try:
+        r1 = min(64, N)
+        _, t3s = _timed(oracle.fold_quant_weights, np.ascontiguousarray(hw[:r1]), s)
+        r1x = min(64, M)
+        _, t4s = _timed(oracle.smooth_quant_act, np.ascontiguousarray(hx[:r1x]), s)
+        r5, c5 = min(4, M), min(512, N)
+        _, t5s = _timed(oracle.gemm_i8, np.ascontiguousarray(xq[:r5]), np.ascontiguousarray(wq[:c5]))
+    finally:
+        oracle.set_num_threads(threads)
+    one = {"a3_gbs": r1 * K * (ies + 1) / t3s / 1e9, "a4_gbs": r1x * K * (ies + 1) / t4s / 1e9,
+           "a5_tops": 2.0 * r5 * c5 * K / t5s / 1e12,
+           "slices": f"a3 {r1} rows, a4 {r1x} rows, a5 {r5} x {c5} outputs (K={K})"}
+    total = t1x + t1w + t2 + t3 + t4 + t5_full
+    tops = 2.0 * M * N * K / total / 1e12
+    desc = (f"oracle per stage on the full tensors (a1 over {hc.shape[0]} calibration tokens and W, a2, a3 over "
+            f"W [{N} x {K}], a4 over X [{M} x {K}]) and a5 on the first {rows} tokens, extrapolated to {M}; "
+            f"value = 2*{M}*{N}*{K} ops / (a1 + a2 + a3 + a4 + a5 extrapolated)")
+    return {"stages": {k: {kk: (round(vv, 6) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                       for k, v in st.items()},
+            "one_thread": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in one.items()}}, tops, desc
+
+
+def oracle_slice(x: torch.Tensor, w: torch.Tensor, alpha: float, tokens: int, rows: int):
+    """The whole path (a1..a5) on a tokens x rows slice (full K) -> seconds."""
     import oracle
     hx = synth.host_array(x[:tokens])
     hw = synth.host_array(w[:rows])
-    K = x.shape[1]
-    ops = 2.0 * tokens * rows * K
-    n, t0 = 0, time.perf_counter()
-    while True:
-        oracle.linear(hx, hw, alpha)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    per = el / n
-    desc = (f"whole path (a1..a5) on a {tokens}-token x {rows}-output-channel slice of the workload "
-            f"(K={K}), {n} repetitions in {el:.1f} s; value = 2*{tokens}*{rows}*{K} int8 ops per slice / time")
-    return ops / per / 1e12, oracle.num_threads(), desc, per
+    t0 = time.perf_counter()
+    oracle.linear(hx, hw, alpha)
+    return time.perf_counter() - t0
 
 
 # ------------------------------------------------------------------ our arm
 def workload_inputs(name: str, decode_m: int):
-    """(workload, x, w, alpha, out bytes) for a workload name; mlp_decode_7b
-    takes its token count from --decode-m and uses the gate projection."""
+    """(workload, x, w, calibration tensor or None) for a workload name;
+    mlp_decode_7b takes its token count from --decode-m and uses the gate
+    projection; down_prefill_70b calibrates on its 16 batches of 2048 tokens."""
     wl = synth.WORKLOADS[name]
+    xcal = None
     if name == "mlp_decode_7b":
         x, w = synth.make_decode(decode_m, "gate")
     else:
         x, w = synth.make(name)
-    return wl, x, w
+    if name == "down_prefill_70b":
+        xcal = torch.cat(list(synth.calibration_batches(name)))
+    return wl, x, w, xcal
 
 
 VARIANTS = {
-    "smoothquant": "a1(X)+a1(W) in one launch, a2, a3+a4 in one launch, a5: per-token dynamic activation "
-                   "scales (O1)",
+    "smoothquant": "a1(calibration X)+a1(W) in one launch, a2, a3 and a4 (one launch where the streamed row kernel "
+                   "takes both tensors), a5: per-token dynamic activation scales (O1)",
     "smoothquant_steps": "a1(X) a1(W) a2 a3 a4 a5, one launch per step (per-step timings)",
     "per_tensor_dynamic": "a1(X) a1(W) a2 a3, per-tensor range of X/s, per-tensor codes, a5 (O2)",
     "per_tensor_static": "a1(X) a1(W) a2 a3, static range from the calibration maxima, per-tensor codes, a5 (O3)",
@@ -222,11 +304,19 @@ ACT_QUANT_STAGES = ("a4_smooth_quant_x", "a34_fold_smooth_quant_wx", "quant_per_
 SPLIT_THRESHOLD = 6.0  # outlier channels: calibration maximum >= 6 (the synthetic outliers are 20-80x)
 
 
-def build_step(variant, sq, wl, x, w, dev, stream):
+def pair_fits(K: int) -> bool:
+    """Whether the streamed row kernel takes a3 and a4 in one launch at this K
+    (both multiplier tables beside the ring); at K = 28672 they do not, and the
+    pair call makes the two launches, so the step lists them separately."""
+    return K <= 16384
+
+
+def build_step(variant, sq, wl, x, w, xcal, dev, stream):
     """Buffers and the ordered stages of one step: [(name, callable, algorithmic
     bytes, ops)]. Every callable is one C ABI call on `stream`."""
     M, K = x.shape
     N = w.shape[0]
+    C = xcal.shape[0]
     in_es = x.element_size()
     out_es = torch.empty(0, dtype=wl.out_dtype).element_size()
     maxima = torch.zeros(2 * K + 4, dtype=torch.float32, device=dev)   # xmax | wmax | amax, cleared per step
@@ -240,6 +330,9 @@ def build_step(variant, sq, wl, x, w, dev, stream):
     gws = sq.gemm_workspace(M, N, K, dev)
     ops = 2.0 * M * N * K
     gemm_bytes = M * K + N * K + M * 4 + N * 4 + M * N * out_es
+    a3_bytes = N * K * in_es + K * 4 + N * K + N * 4
+    act_bytes = M * K * in_es + K * 4 + M * K + M * 4
+    bufs = dict(maxima=maxima, xmax=xmax, wmax=wmax, s=s, wq=wq, wsc=wsc, xq=xq, xsc=xsc, y=y, gws=gws)
     st = []
     if variant == "alpha_search":
         alphas = list(synth.DOWN_70B_ALPHAS)
@@ -253,42 +346,47 @@ def build_step(variant, sq, wl, x, w, dev, stream):
             errs, best = sq.sq_alpha_search(x, w, alphas, workspace=sws, stream=stream)
             result.update(errors=[round(e, 6) for e in errs], best_alpha=best)
         st.append(("alpha_search", search, once + len(alphas) * per_alpha, len(alphas) * ops))
-        return maxima, st, {"alphas": alphas, "search": result,
-                            "note": "the call synchronizes its stream; ops = int8 GEMM ops over all alphas"}
+        return bufs, st, {"alphas": alphas, "search": result,
+                          "note": "the call synchronizes its stream; ops = int8 GEMM ops over all alphas"}
+    a1_pair = ("a1_calibrate_xw", lambda: sq.sq_calibrate_absmax_pair(xcal, w, xmax, wmax, stream=stream),
+               (C + N) * K * in_es + 2 * K * 4, 0)
+    a2 = ("a2_smooth_factors", lambda: sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream),
+          3 * K * 4, 0)
+    a5 = ("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm(xq, xsc, wq, wsc, y=y, workspace=gws, stream=stream),
+          gemm_bytes, ops)
     if variant == "fp8":
         wq8 = torch.empty((N, K), dtype=torch.uint8, device=dev)
         xq8 = torch.empty((M, K), dtype=torch.uint8, device=dev)
-        st.append(("a1_calibrate_xw", lambda: sq.sq_calibrate_absmax_pair(x, w, xmax, wmax, stream=stream),
-                   (M + N) * K * in_es + 2 * K * 4, 0))
-        st.append(("a2_smooth_factors", lambda: sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream),
-                   3 * K * 4, 0))
+        st += [a1_pair, a2]
         st.append(("a34_fold_smooth_quant_wx_e4m3",
                    lambda: sq.sq_fold_smooth_quant_pair_e4m3(w, x, s, wq=wq8, w_scale=wsc, xq=xq8, x_scale=xsc,
                                                              stream=stream),
                    (N + M) * K * in_es + K * 4 + (N + M) * K + (N + M) * 4, 0))
         st.append(("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm_e4m3(xq8, xsc, wq8, wsc, y=y, stream=stream),
                    gemm_bytes, ops))
-        return maxima, st, {"note": "FP8 E4M3 codes; the GEMM kernel is the paired-SM tcgen05 kernel with "
-                                    "kind::f8f6f4 operands"}
+        return bufs, st, {"note": "FP8 E4M3 codes; the GEMM kernel is the paired-SM tcgen05 kernel with "
+                                  "kind::f8f6f4 operands"}
     if variant == "smoothquant":
-        st.append(("a1_calibrate_xw", lambda: sq.sq_calibrate_absmax_pair(x, w, xmax, wmax, stream=stream),
-                   (M + N) * K * in_es + 2 * K * 4, 0))
-        st.append(("a2_smooth_factors", lambda: sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream),
-                   3 * K * 4, 0))
-        st.append(("a34_fold_smooth_quant_wx",
-                   lambda: sq.sq_fold_smooth_quant_pair(w, x, s, wq=wq, w_scale=wsc, xq=xq, x_scale=xsc,
-                                                        stream=stream),
-                   (N + M) * K * in_es + K * 4 + (N + M) * K + (N + M) * 4, 0))
-        st.append(("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm(xq, xsc, wq, wsc, y=y, workspace=gws, stream=stream),
-                   gemm_bytes, ops))
-        return maxima, st, {}
-    st.append(("a1_calibrate_x", lambda: sq.sq_calibrate_absmax(x, xmax, stream=stream), M * K * in_es + K * 4, 0))
+        st += [a1_pair, a2]
+        if pair_fits(K):
+            st.append(("a34_fold_smooth_quant_wx",
+                       lambda: sq.sq_fold_smooth_quant_pair(w, x, s, wq=wq, w_scale=wsc, xq=xq, x_scale=xsc,
+                                                            stream=stream),
+                       (N + M) * K * in_es + K * 4 + (N + M) * K + (N + M) * 4, 0))
+        else:
+            st.append(("a3_fold_quant_w", lambda: sq.sq_fold_quant_weights(w, s, wq=wq, w_scale=wsc, stream=stream),
+                       a3_bytes, 0))
+            st.append(("a4_smooth_quant_x", lambda: sq.sq_smooth_quant_act(x, s, xq=xq, x_scale=xsc, stream=stream),
+                       act_bytes, 0))
+        st.append(a5)
+        return bufs, st, {}
+    st.append(("a1_calibrate_x", lambda: sq.sq_calibrate_absmax(xcal, xmax, stream=stream), C * K * in_es + K * 4, 0))
     if variant == "split":
         keep = torch.empty(K, dtype=torch.float32, device=dev)
         idx = torch.empty(K, dtype=torch.int32, device=dev)
         count = torch.empty(1, dtype=torch.int32, device=dev)
         # the outlier set is static: its size is fixed once, from this workload's calibration
-        sq.sq_calibrate_absmax(x, xmax, stream=stream)
+        sq.sq_calibrate_absmax(xcal, xmax, stream=stream)
         _, _, c0 = sq.sq_outlier_split(xmax, SPLIT_THRESHOLD, stream=stream)
         n_out = int(c0.item())
         ld = max(4, (n_out + 3) // 4 * 4)
@@ -297,10 +395,8 @@ def build_step(variant, sq, wl, x, w, dev, stream):
 
         st.append(("outlier_split", lambda: sq.sq_outlier_split(xmax, SPLIT_THRESHOLD, keep=keep, idx=idx, count=count,
                                                                 stream=stream), K * 4 * 2 + K * 4, 0))
-        st.append(("quant_bulk_w", lambda: sq.sq_quant_bulk(w, keep, q=wq, scale=wsc, stream=stream),
-                   N * K * in_es + K * 4 + N * K + N * 4, 0))
-        st.append(("quant_bulk_x", lambda: sq.sq_quant_bulk(x, keep, q=xq, scale=xsc, stream=stream),
-                   M * K * in_es + K * 4 + M * K + M * 4, 0))
+        st.append(("quant_bulk_w", lambda: sq.sq_quant_bulk(w, keep, q=wq, scale=wsc, stream=stream), a3_bytes, 0))
+        st.append(("quant_bulk_x", lambda: sq.sq_quant_bulk(x, keep, q=xq, scale=xsc, stream=stream), act_bytes, 0))
         st.append(("gather_x", lambda: sq.sq_gather_columns(x, idx, n_out, ld, out=xo, stream=stream),
                    M * n_out * in_es + M * ld * 4, 0))
         st.append(("gather_w", lambda: sq.sq_gather_columns(w, idx, n_out, ld, out=wo, stream=stream),
@@ -308,13 +404,11 @@ def build_step(variant, sq, wl, x, w, dev, stream):
         st.append(("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm_split(xq, xsc, wq, wsc, xo, wo, y=y, workspace=gws,
                                                                   stream=stream),
                    gemm_bytes + (M + N) * ld * 4, ops))
-        return maxima, st, {"outlier_channels": n_out, "ld": ld, "threshold": SPLIT_THRESHOLD}
+        return bufs, st, {"outlier_channels": n_out, "ld": ld, "threshold": SPLIT_THRESHOLD}
     st.append(("a1_calibrate_w", lambda: sq.sq_calibrate_absmax(w, wmax, stream=stream), N * K * in_es + K * 4, 0))
-    st.append(("a2_smooth_factors", lambda: sq.sq_smooth_factors(xmax, wmax, wl.alpha, 1e-8, s=s, stream=stream),
-               3 * K * 4, 0))
+    st.append(a2)
     st.append(("a3_fold_quant_w", lambda: sq.sq_fold_quant_weights(w, s, wq=wq, w_scale=wsc, stream=stream),
-               N * K * in_es + K * 4 + N * K + N * 4, 0))
-    act_bytes = M * K * in_es + K * 4 + M * K + M * 4
+               a3_bytes, 0))
     extra = {}
     if variant == "smoothquant_steps":
         st.append(("a4_smooth_quant_x", lambda: sq.sq_smooth_quant_act(x, s, xq=xq, x_scale=xsc, stream=stream),
@@ -341,9 +435,46 @@ def build_step(variant, sq, wl, x, w, dev, stream):
                    act_bytes, 0))
         extra = {"norm_eps": 1e-5, "note": "x plays the hidden state; s from its maxima (kernel cost is "
                                            "independent of the values of s)"}
-    st.append(("a5_w8a8_gemm", lambda: sq.sq_w8a8_gemm(xq, xsc, wq, wsc, y=y, workspace=gws, stream=stream),
-               gemm_bytes, ops))
-    return maxima, st, extra
+    st.append(a5)
+    return bufs, st, extra
+
+
+def int8_probe(sq, dev, stream, clk, launches=PROBE_LAUNCHES, iters=PROBE_ITERS):
+    """The int8 tensor-core rate (sq_probe_tensor_int8), median over launches
+    with CUDA events on the launching stream -> dict."""
+    clk.mark("probe")
+    times, ops = [], 0.0
+    for i in range(launches + 3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ops = sq.sq_probe_tensor_int8(iters, stream=stream)
+        b.record(stream)
+        b.synchronize()
+        if i >= 3:
+            times.append(a.elapsed_time(b))
+    ms = median(times)
+    return {"tops": ops / (ms * 1e-3) / 1e12, "ms": ms, "ops_per_launch": ops, "launches": launches,
+            "instruction": "tcgen05.mma.cta_group::2.kind::i8 256x256x32 from shared memory, every SM pair"}
+
+
+def int_mm_probe(dev, stream, n=8192, reps=10):
+    """torch._int_mm (a library int8 GEMM) at n^3, best of `reps`, as context."""
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        for _ in range(2):
+            torch._int_mm(a, b)
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            torch._int_mm(a, b)
+            e1.record(stream)
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return {"tops": 2.0 * n ** 3 / (best * 1e-3) / 1e12, "ms": round(best, 4), "shape": f"{n}^3"}
+    except Exception as e:  # pragma: no cover - depends on the box
+        return {"unavailable": repr(e)[:200]}
 
 
 def run_ours(args, world, rank, local):
@@ -351,15 +482,17 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     init_dist(world, "nccl")
-    wl, x_cpu, w_cpu = workload_inputs(args.workload, args.decode_m)
+    wl, x_cpu, w_cpu, xcal_cpu = workload_inputs(args.workload, args.decode_m)
     M, K = x_cpu.shape
     N = w_cpu.shape[0]
     x = x_cpu.to(dev)
     w = w_cpu.to(dev)
+    xcal = x if xcal_cpu is None else xcal_cpu.to(dev)
     in_es, out_es = x_cpu.element_size(), torch.empty(0, dtype=wl.out_dtype).element_size()
     stream = torch.cuda.current_stream(dev)
 
-    maxima, stages, variant_info = build_step(args.variant, sq, wl, x, w, dev, stream)
+    bufs, stages, variant_info = build_step(args.variant, sq, wl, x, w, xcal, dev, stream)
+    maxima = bufs["maxima"]
     names = [n for n, _, _, _ in stages]
     nst = len(stages)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -371,7 +504,6 @@ def run_ours(args, world, rank, local):
         # kernel would pay for.
         flush.zero_()
         flush_read.amax()
-    launches_per_step = nst
 
     def step(ev=None):
         maxima.zero_()
@@ -388,49 +520,57 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("device status error during warm-up")
 
     # Timed region: K steps with one event pair each (no events between the
-    # kernels, so consecutive launches may overlap as they do in use).
+    # kernels, so consecutive launches overlap as they do in use: every kernel
+    # is launched with programmatic dependent launch).
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     # A second, instrumented pass (events between the kernels) gives each
     # kernel's duration for the kernel table and the roofline.
-    n_inst = min(args.steps, 200)
+    n_inst = max(args.steps, args.kernel_steps)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(n_inst)]
-    barrier(world)
-    torch.cuda.synchronize(dev)
+    sweep = None
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        clk.mark("steps")
         for i in range(args.steps):
             flush_l2()
             step_ev[i][0].record(stream)
             step()
             step_ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark("between")
         barrier(world)
+        clk.mark("kernels")
         for i in range(n_inst):
             flush_l2()
             step(events[i])
         torch.cuda.synchronize(dev)
+        clk.mark("between")
+        if args.variant == "smoothquant" and args.sweep_steps > 0 and wl.name == "down_prefill_70b":
+            clk.mark("sweep")
+            sweep = alpha_sweep(sq, bufs, stages, x, w, stream, flush_l2, args.sweep_steps)
+            clk.mark("between")
+        probe = int8_probe(sq, dev, stream, clk) if M > 16 else None
+        clk.mark("between")
     barrier(world)
     status = sq.sq_get_status(stream)
     if status != sq.SQ_OK:
         raise RuntimeError(f"device status {status} after the timed region")
 
-    step_ms = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
-    per_kernel = {n: 0.0 for n in names}
-    inst_step_ms = 0.0
-    for ev in events:
-        inst_step_ms += ev[0].elapsed_time(ev[nst])
-        for j, n in enumerate(names):
-            per_kernel[n] += ev[j].elapsed_time(ev[j + 1])
-    inst_step_ms /= n_inst
-    per_kernel = {n: v / n_inst for n, v in per_kernel.items()}
+    step_times = [a.elapsed_time(b) for a, b in step_ev]
+    step_ms = median(step_times)
+    per_kernel = {n: median([ev[j].elapsed_time(ev[j + 1]) for ev in events]) for j, n in enumerate(names)}
+    inst_step_ms = median([ev[0].elapsed_time(ev[nst]) for ev in events])
     step_ms_max = max_over_ranks(step_ms, world, dev)
     ops = 2.0 * M * N * K
     value = world * ops / (step_ms_max * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    int8_peak = bf16_peak * INT8_OVER_BF16
+    int8_from_bf16 = bf16_peak * INT8_OVER_BF16
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    int8_peak = probe["tops"] if probe else int8_from_bf16
     kb = {n: b for n, _, b, _ in stages}
     kernels = {}
     for n in names:
@@ -441,8 +581,11 @@ def run_ours(args, world, rank, local):
         if n == "a5_w8a8_gemm":
             tops = ops / (ms * 1e-3) / 1e12
             entry.update({"tops": round(tops, 1), "tensor_frac": round(tops / int8_peak, 3),
+                          "tensor_frac_of_bf16x2": round(tops / int8_from_bf16, 3),
                           "tensor_frac_of_spec": round(tops / SPEC_INT8_TOPS, 3)})
         kernels[n] = entry
+    clocks_k = clk.summary({"kernels"})
+    clocks_p = clk.summary({"probe"})
     if args.variant == "alpha_search":
         ms = per_kernel["alpha_search"]
         n_a = len(variant_info["alphas"])
@@ -454,23 +597,29 @@ def run_ours(args, world, rank, local):
                     "traffic": None, "peak_source": f"{peak_src}: hbm_gbs",
                     "algorithmic_bytes_per_launch": kb["alpha_search"]}
         kernels["alpha_search"]["per_alpha_ms"] = round(ms / n_a, 4)
-    else:
+    elif M > 16:
         gemm_ms = per_kernel["a5_w8a8_gemm"]
         achieved = ops / (gemm_ms * 1e-3) / 1e12
-    default_gemm = args.variant != "split"
-    if args.variant == "alpha_search":
-        pass
-    elif M > 16:
+        default_gemm = args.variant not in ("split", "fp8")
         roofline = {"bound": "tensor", "kernel": ("gemm_pair_kernel (a5, paired-SM tcgen05)" if M > 128
                                                   else "gemm_tiled_kernel (a5)")
                     + (", FP8 E4M3 operands" if args.variant == "fp8" else ""),
                     "achieved": round(achieved, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
                     "frac": round(achieved / int8_peak, 4),
-                    "traffic": load_traffic() if (M > 128 and default_gemm and args.variant != "fp8") else None,
-                    "peak_source": f"{peak_src}: bf16 {bf16_peak} TFLOP/s (burst) x {INT8_OVER_BF16} nominal "
-                                   f"int8/bf16 ratio",
+                    "traffic": load_traffic(args.workload) if (M > 128 and default_gemm) else None,
+                    "peak_source": ("measured int8: sq_probe_tensor_int8 in this run (median of "
+                                    f"{probe['launches']} launches of {probe['ms']:.3f} ms), SM clock median "
+                                    f"{clocks_p.get('sm_mhz')} MHz during the probe, "
+                                    f"{clocks_k.get('sm_mhz')} MHz during the kernel pass" if probe else
+                                    f"{peak_src}: bf16 x {INT8_OVER_BF16}"),
+                    "peak_bf16x2": round(int8_from_bf16, 1),
+                    "frac_of_bf16x2": round(achieved / int8_from_bf16, 4),
+                    "bf16x2_source": f"{peak_src}: bf16 {bf16_peak} TFLOP/s (burst) x {INT8_OVER_BF16} nominal "
+                                     f"int8/bf16 ratio",
+                    "peak_spec": SPEC_INT8_TOPS, "frac_of_spec": round(achieved / SPEC_INT8_TOPS, 4),
                     "algorithmic_ops_per_launch": ops}
     else:
+        gemm_ms = per_kernel["a5_w8a8_gemm"]
         gbs = kb["a5_w8a8_gemm"] / (gemm_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "kernel": "gemm_stream_kernel (a5, split-K weight streaming)",
                     "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
@@ -504,66 +653,142 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": x_cpu.numel() * in_es + w_cpu.numel() * in_es,
                "d2h_bytes_per_step": M * N * out_es,
                "api": "sq_linear (C ABI) with pinned host buffers, calls back to back (each call's input copies "
-                      "overlap the previous call's GEMM and output copy)"}
+                      "overlap the previous call's GEMM and output copy); sq_linear calibrates on its own batch"}
+        del xh, wh, yh, lws
+
+    int_mm = int_mm_probe(dev, stream) if (M > 16 and args.int_mm) else None
 
     cpu_baseline = None
-    if rank == 0 and world == 1 and args.cpu_seconds > 0 and args.variant == "smoothquant":
-        v, cores, desc, _ = oracle_sample(x_cpu, w_cpu, wl.alpha, args.cpu_seconds)
-        cpu_baseline = {"value": round(v, 5), "unit": "TOPS", "cores": cores, "kind": "oracle",
-                        "sample": desc}
+    if rank == 0 and world == 1 and args.cpu_baseline and args.variant == "smoothquant":
+        import oracle
+        per, tops_cpu, desc = oracle_stages(x_cpu, w_cpu, wl.alpha, xcal_cpu)
+        cpu_baseline = {"value": round(tops_cpu, 6), "unit": "TOPS", "cores": oracle.num_threads(),
+                        "kind": "oracle", "sample": desc, "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+                        **per}
+        if args.workload != "qkv_prefill_7b":
+            _, xq7, wq7, _ = workload_inputs("qkv_prefill_7b", 16)
+            per7, tops7, _ = oracle_stages(xq7, wq7, synth.WORKLOADS["qkv_prefill_7b"].alpha)
+            cpu_baseline["qkv_prefill_7b"] = {"tops": round(tops7, 6), **per7}
 
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
         return None
-    return {
+    launches = nst   # one launch of this library per stage
+    out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-        "data": "synthetic (seeded outlier-bearing activations, N(0,1/64) weights)",
+        "data": "synthetic (seeded outlier-bearing activations, N(0, 1/sqrt(K)) weights)",
         "config": {"workload": args.workload, "M": M, "N": N, "K": K,
                    "in_dtype": str(x_cpu.dtype).replace("torch.", ""),
                    "out_dtype": str(wl.out_dtype).replace("torch.", ""),
-                   "alpha": wl.alpha, "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
+                   "alpha": wl.alpha,
+                   "calibration": (f"{xcal.shape[0] // synth.DOWN_70B_CALIB_TOKENS} batches x "
+                                   f"{synth.DOWN_70B_CALIB_TOKENS} tokens, resident, one launch"
+                                   if xcal_cpu is not None else "the step's own batch"),
+                   "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "variant": args.variant, "step": VARIANTS[args.variant] + ", one stream", **variant_info,
-                   "timing": f"{args.steps} steps with one CUDA event pair each (the value); per-kernel times "
-                             f"from {n_inst} further steps with events between the kernels "
-                             f"({round(inst_step_ms, 5)} ms per step there)"},
+                   "timing": f"value: median of {args.steps} steps with one CUDA event pair each (mean "
+                             f"{round(sum(step_times) / len(step_times), 5)} ms); kernel table: medians over "
+                             f"{n_inst} further steps with events between the kernels (the step there "
+                             f"{round(inst_step_ms, 5)} ms: events between kernels stop the launches' overlap)"},
         "act_quant_gbs": next((kernels[n]["gbs"] for n in ACT_QUANT_STAGES if n in kernels), None),
         "act_quant_gbs_from": next((n for n in ACT_QUANT_STAGES if n in kernels), None),
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary({"steps", "kernels", "sweep"}),
+        "clocks_by_phase": {p: clk.summary({p}) for p in ("steps", "kernels", "sweep", "probe")},
     }
+    if probe:
+        out["int8_probe"] = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in probe.items()}
+    if int_mm:
+        out["int_mm_context"] = int_mm
+    if sweep:
+        out["alpha_sweep"] = sweep
+    return out
+
+
+def alpha_sweep(sq, bufs, stages, x, w, stream, flush_l2, steps):
+    """Per alpha in {0.25, 0.5, 0.75}: a2, a3, a4 and a5 after the step's
+    calibration (the maxima of the last step stay in place), timed per stage
+    with CUDA events, medians over `steps` repetitions; plus the codes'
+    agreement check that the three alphas give three different weight sets."""
+    xmax, wmax, s = bufs["xmax"], bufs["wmax"], bufs["s"]
+    wq, wsc, xq, xsc, y, gws = bufs["wq"], bufs["wsc"], bufs["xq"], bufs["xsc"], bufs["y"], bufs["gws"]
+    # calibration once (the sweep reuses it)
+    bufs["maxima"].zero_()
+    stages[0][1]()
+    M, K = x.shape
+    N = w.shape[0]
+    ops = 2.0 * M * N * K
+    out = {}
+    w_checksums = []
+    for a in synth.DOWN_70B_ALPHAS:
+        fns = [("a2", lambda: sq.sq_smooth_factors(xmax, wmax, a, 1e-8, s=s, stream=stream)),
+               ("a3", lambda: sq.sq_fold_quant_weights(w, s, wq=wq, w_scale=wsc, stream=stream)),
+               ("a4", lambda: sq.sq_smooth_quant_act(x, s, xq=xq, x_scale=xsc, stream=stream)),
+               ("a5", lambda: sq.sq_w8a8_gemm(xq, xsc, wq, wsc, y=y, workspace=gws, stream=stream))]
+        times = {n: [] for n, _ in fns}
+        tot = []
+        for i in range(steps + 2):
+            flush_l2()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+            for j, (_, fn) in enumerate(fns):
+                ev[j].record(stream)
+                fn()
+            ev[-1].record(stream)
+            ev[-1].synchronize()
+            if i >= 2:
+                for j, (n, _) in enumerate(fns):
+                    times[n].append(ev[j].elapsed_time(ev[j + 1]))
+                tot.append(ev[0].elapsed_time(ev[-1]))
+        w_checksums.append(float(wsc.double().sum().item()))
+        ms = median(tot)
+        out[str(a)] = {"ms": round(ms, 5), "tops": round(ops / (ms * 1e-3) / 1e12, 1),
+                       **{f"{n}_ms": round(median(v), 5) for n, v in times.items()}}
+    out["distinct_weight_scales"] = len(set(w_checksums)) == len(w_checksums)
+    out["note"] = (f"a2..a5 per alpha after the step's calibration, medians of {steps} repetitions with events "
+                   "between the stages, L2 flushed before each")
+    return out
 
 
 # ------------------------------------------------------------------ reference arm
 def run_reference(args, world, rank):
     """The oracle (plain C on the host cores) on this workload, as the
-    reference arm: each step is one bounded sample of the workload."""
+    reference arm: each step is one bounded sample of the workload (the whole
+    path on a slice of tokens x output channels, full K)."""
     if rank != 0:
         return None
-    wl, x_cpu, w_cpu = workload_inputs(args.workload, args.decode_m)
-    M, K = x_cpu.shape
-    N = w_cpu.shape[0]
+    import oracle
+    wl = synth.WORKLOADS[args.workload]
+    if args.workload == "mlp_decode_7b":
+        x_cpu, w_cpu = synth.make_decode(args.decode_m, "gate")
+    else:
+        # the slice the arm times is all it needs: draw only those rows
+        x_cpu = synth.activations(min(64, wl.T), wl.K, wl.outliers, wl.seed, wl.in_dtype)
+        w_cpu = synth.weights(min(256, wl.N), wl.K, wl.w_std, wl.seed, wl.in_dtype)
+    if args.workload == "mlp_decode_7b":
+        M, K, N = x_cpu.shape[0], x_cpu.shape[1], w_cpu.shape[0]
+    else:
+        M, K, N = wl.T, wl.K, wl.N
     budget = max(0.002, args.reference_budget_s / max(1, args.steps + args.warmup))
-    # size the slice so one step stays within the budget
-    tokens, rows = min(64, M), min(256, N)
-    _, _, _, per = oracle_sample(x_cpu, w_cpu, wl.alpha, 0.0, tokens, rows)
+    tokens, rows = min(64, x_cpu.shape[0]), min(256, w_cpu.shape[0])
+    per = oracle_slice(x_cpu, w_cpu, wl.alpha, tokens, rows)
     while per > budget and tokens > 1:
         tokens //= 2
         per /= 2
     for _ in range(args.warmup):
-        oracle_sample(x_cpu, w_cpu, wl.alpha, 0.0, tokens, rows)
-    t0 = time.perf_counter()
+        oracle_slice(x_cpu, w_cpu, wl.alpha, tokens, rows)
+    el = 0.0
     for _ in range(args.steps):
-        oracle_sample(x_cpu, w_cpu, wl.alpha, 0.0, tokens, rows)
-    el = time.perf_counter() - t0
+        el += oracle_slice(x_cpu, w_cpu, wl.alpha, tokens, rows)
     ops = 2.0 * tokens * rows * K
     value = ops * args.steps / el / 1e12
-    import oracle
     desc = (f"oracle whole path (a1..a5) on a {tokens}-token x {rows}-output-channel slice of the "
-            f"workload per step (K={K}); value = int8 ops of the slice / time")
+            f"workload per step (K={K}); value = int8 ops of the slice / time; {cpu_model()}, "
+            f"{os.cpu_count()} logical CPUs")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
@@ -580,17 +805,23 @@ def run_reference(args, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=WORKLOAD,
-                    help="the measured configuration is the 7B QKV prefill; the others are for profiling")
+                    help="the measured configuration is the 70B down projection prefill; the others are for "
+                         "profiling")
     ap.add_argument("--decode-m", type=int, default=16, choices=synth.DECODE_MS)
     ap.add_argument("--variant", choices=sorted(VARIANTS), default="smoothquant",
                     help="the measured path is smoothquant (per-token O1); the others measure the other "
                          "activation granularities, the norm-folded form and the outlier decomposition")
-    ap.add_argument("--e2e-steps", type=int, default=10, help="steps of the end-to-end measurement")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
+    ap.add_argument("--kernel-steps", type=int, default=100, help="steps of the instrumented (per-kernel) pass")
+    ap.add_argument("--sweep-steps", type=int, default=10, help="repetitions per alpha of the alpha sweep")
+    ap.add_argument("--e2e-steps", type=int, default=5, help="steps of the end-to-end measurement")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false",
+                    help="skip the oracle's per-stage timing on the host cores")
+    ap.add_argument("--no-int-mm", dest="int_mm", action="store_false",
+                    help="skip the torch._int_mm context figure")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -52,7 +52,9 @@ typedef enum sq_status {
     SQ_ERR_UNSUPPORTED = 2,  /* K not a multiple of 16, misaligned pointer, unsupported dtype
                                 or size */
     SQ_ERR_CUDA = 3,         /* a CUDA runtime call failed; see sq_last_error_string() */
-    SQ_ERR_TIMEOUT = 4       /* a kernel's bounded wait ran out (reported by sq_get_status) */
+    SQ_ERR_TIMEOUT = 4,      /* a kernel's bounded wait ran out (reported by sq_get_status) */
+    SQ_ERR_BOUNDS = 5        /* debug builds only (-DSQ_DEBUG): a kernel's index check found a store
+                                outside its buffer and skipped it (reported by sq_get_status) */
 } sq_status;
 
 typedef enum sq_dtype {
@@ -298,12 +300,15 @@ sq_status sq_w8a8_gemm_split(const int8_t* xq, const float* x_scale, const int8_
  * weight-streaming path), but keeps that path's scratch (partial sums and
  * completion counters) in a fixed array inside the library instead of a
  * caller workspace, and allocates nothing.
- *   Limits: 1 <= M <= 16, M * N <= 262,144 and N <= 262,144 (1 MiB + 32 KiB of
- *   scratch, held by every GPU that loads the library until the process
- *   exits); larger sizes return SQ_ERR_UNSUPPORTED with a message. M == 0 or
- *   N == 0 is a no-op.
- *   The first call on a device looks up the scratch array's device address;
- *   make that first call before capturing any stream into a CUDA graph.
+ *   Limits: 1 <= M <= 16 and M * N <= 262,144 (1 MiB + 32 KiB of scratch,
+ *   held by every GPU that loads the library until the process exits); larger
+ *   sizes return SQ_ERR_UNSUPPORTED with a message. M == 0 or N == 0 is a
+ *   no-op.
+ *   The first call on a device looks up the scratch array's device address and
+ *   keeps it for the life of the process; make that first call before
+ *   capturing any stream into a CUDA graph. After cudaDeviceReset on that
+ *   device the kept address is stale: do not call this function on that
+ *   device again in the same process.
  *   Each call clears the part of the scratch it uses (cudaMemsetAsync on
  *   `stream`) before its kernel. All calls on a device share the one array:
  *   calls that overlap on the GPU (different streams, no ordering between
@@ -312,6 +317,11 @@ sq_status sq_w8a8_gemm_split(const int8_t* xq, const float* x_scale, const int8_
 sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* x_scale, const int8_t* wq,
                                const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,
                                sq_dtype out_dt, sq_stream_t stream);
+/* Test hook for the entry point above: fills the current device's whole
+ * scratch array with a non-zero byte pattern on `stream`, as a call that
+ * stopped early (a bounded wait that ran out) would leave it, so a test can
+ * check that the next call still starts from a cleared scratch. */
+sq_status sq_selftest_dirty_noalloc_scratch(sq_stream_t stream);
 
 /* ---------------------------------------------------------------- alpha search
  * Per-layer choice of the migration strength: for each candidate alpha the
@@ -323,8 +333,10 @@ sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* x_scale, const int
  * answer": the alpha sweep and its W8A8 error column; "SmoothQuant
  * Explained", "Alpha: how much difficulty to move": the best alpha is
  * model-specific). The maxima (a1) come from x and w once. Y is computed once
- * with cuBLAS (a plain floating-point GEMM: bf16 or fp32 operands, fp32
- * accumulation); the sums of squares are fp64.
+ * by this library's own kernels: for bf16 operands the tcgen05 GEMM with
+ * kind::f16 (every product exact in fp32, the sum accumulated in fp32 in the
+ * tensor core's order), for fp32 operands a CUDA-core GEMM (a chain of fp32
+ * fused multiply-adds in k order). The sums of squares are fp64.
  *   x [T x K], w [N x K]: dtype in_dt (SQ_F32 or SQ_BF16), device.
  *   alphas [n_alpha] float, HOST, each in [0, 1]; 1 <= n_alpha <= 64.
  *   eps as for sq_smooth_factors.
@@ -394,9 +406,35 @@ sq_status sq_w8a8_gemm_e4m3(const uint8_t* xq, const float* x_scale, const uint8
  *   Zero-fill it once before its first use (it contains the GEMM workspace). */
 size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K, sq_dtype in_dt,
                                 sq_dtype out_dt);
+/* Where sq_linear keeps the layer's intermediates inside its workspace, so a
+ * caller can read or reuse them after the call (the int8 weights and their
+ * scales, say, to run later batches through sq_w8a8_gemm alone): byte offsets
+ * from the workspace base of, in this order,
+ *   [0] xmax [K] float   [1] wmax [K] float   [2] s [K] float
+ *   [3] xq [M x K] int8  [4] x_scale [M] float
+ *   [5] wq [N x K] int8  [6] w_scale [N] float
+ * (7 entries, each a multiple of 256). They hold the last call's values once
+ * that call's work on its stream has completed. Host only (no CUDA call).
+ * Returns SQ_ERR_INVALID_ARG for a negative size or NULL offsets, and
+ * SQ_ERR_UNSUPPORTED for a dtype sq_linear does not take. */
+sq_status sq_linear_workspace_offsets(int64_t M, int64_t N, int64_t K, sq_dtype in_dt,
+                                      sq_dtype out_dt, size_t* offsets);
 sq_status sq_linear(const void* x, const void* w, sq_dtype in_dt, int64_t M, int64_t N,
                     int64_t K, float alpha, float eps, void* y, sq_dtype out_dt,
                     void* workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* ---------------------------------------------------------------- measurement aid
+ * sq_probe_tensor_int8: the int8 tensor-core rate of the current GPU, as a
+ * roofline denominator for the int8 GEMM. The pages state only that integer
+ * tensor cores run at roughly twice the FP16 rate ("SmoothQuant Explained",
+ * "Where it fits"); this measures it. One launch on `stream`: every pair of
+ * SMs issues `iters` x 4 of the prefill GEMM's instruction
+ * (tcgen05.mma.cta_group::2.kind::i8, 256 x 256 x 32) on operands held in
+ * shared memory, with no global-memory traffic. *ops (host, may be NULL)
+ * receives the int8 operations the launch performs (2 per multiply-add); the
+ * caller times the launch (for example with CUDA events on `stream`).
+ * iters in [1, 10^7], else SQ_ERR_INVALID_ARG. Computes nothing else. */
+sq_status sq_probe_tensor_int8(int64_t iters, double* ops, sq_stream_t stream);
 
 /* ---------------------------------------------------------------- status
  * Synchronize `stream`, then return and clear the first error any kernel of

@@ -86,3 +86,37 @@ def freivalds(acc: np.ndarray, xq: np.ndarray, wq: np.ndarray, rounds: int = 3, 
 def oracle_rows(xq: np.ndarray, wq: np.ndarray, rows: np.ndarray) -> np.ndarray:
     """Oracle int32 accumulators for a subset of rows."""
     return oracle.gemm_i8(np.ascontiguousarray(xq[rows]), wq)
+
+
+class Guarded:
+    """A device output buffer with guard bands: `band` bytes of a seeded
+    pattern before and after the buffer proper, which every call writing the
+    buffer must leave as they were (a check for stray writes, in place of a
+    memory checker). `t` is the typed view the call writes; its start is
+    256-byte aligned."""
+
+    def __init__(self, shape, dtype, device, band=4096, seed=0):
+        n = 1
+        for d in shape:
+            n *= d
+        nbytes = n * torch.empty(0, dtype=dtype).element_size()
+        self.band = band
+        self.nbytes = nbytes
+        g = torch.Generator().manual_seed(seed)
+        self.pattern = torch.randint(0, 256, (2 * band,), generator=g, dtype=torch.uint8)
+        tail_pad = (-nbytes) % 256
+        self.raw = torch.empty(band + nbytes + tail_pad + band, dtype=torch.uint8, device=device)
+        self.raw.fill_(0x5A)
+        self.raw[:band] = self.pattern[:band].to(device)
+        self.raw[band + nbytes:band + nbytes + band] = self.pattern[band:].to(device)
+        self.t = self.raw[band:band + nbytes].view(dtype).view(shape)
+
+    def check(self, what: str) -> None:
+        torch.cuda.synchronize()
+        raw = self.raw.cpu()
+        before = raw[:self.band]
+        after = raw[self.band + self.nbytes:self.band + self.nbytes + self.band]
+        for name, got, want in (("before", before, self.pattern[:self.band]),
+                                ("after", after, self.pattern[self.band:])):
+            bad = torch.nonzero(got != want).flatten()
+            assert bad.numel() == 0, f"{what}: {bad.numel()} guard bytes changed {name} the buffer, first at {bad[:4].tolist()}"

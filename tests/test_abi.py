@@ -95,3 +95,12 @@ def test_workspace_sizes(sq):
     assert sq.sq_w8a8_gemm_workspace_size(0, 16, 16) == 0
     need = sq.sq_linear_workspace_size(64, 1024, 1024, sq.torch.float32, sq.torch.float32)
     assert need >= 64 * 1024 + 1024 * 1024 + 3 * 4096
+
+
+def test_library_links_no_library_gemm(sq):
+    """Every step and the alpha search's float product run in libsq's own
+    kernels: the library needs no BLAS."""
+    out = subprocess.run(["readelf", "-d", sq.LIB_PATH], capture_output=True, text=True).stdout
+    needed = re.findall(r"\(NEEDED\)\s+Shared library: \[([^\]]+)\]", out)
+    assert needed, out[:500]
+    assert not [n for n in needed if "blas" in n.lower()], needed

@@ -1,6 +1,6 @@
 """Build libsq.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m w8a8_post_quantization_calibrate_b200.build [--force] [--verbose]
+    python -m w8a8_post_quantization_calibrate_b200.build [--force] [--verbose] [--debug]
 
 The library is one translation unit (csrc/sq_lib.cu includes the others) built
 with -gencode arch=compute_100a,code=sm_100a and -lineinfo. No GPU is needed to
@@ -19,6 +19,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsq.so")
+# the same sources with -DSQ_DEBUG: index checks before the kernels' unguarded
+# stores, reported through the status word (never a trap)
+LIB_DEBUG = os.path.join(PKG, "libsq_debug.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -35,31 +38,31 @@ def sources() -> list[str]:
                   glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(INCLUDE, "sq.h")])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
     cmd = [nvcc(), "-std=c++17", "-O3", "-lineinfo", *ARCH_FLAGS,
-           "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC,
-           "-o", LIB + ".tmp", os.path.join(CSRC, "sq_lib.cu"), "-lcublas"]
+           "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC, *(["-DSQ_DEBUG"] if debug else []),
+           "-o", lib + ".tmp", os.path.join(CSRC, "sq_lib.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libsq.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

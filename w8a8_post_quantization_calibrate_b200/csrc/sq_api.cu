@@ -285,6 +285,27 @@ size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K, sq_dtype in_dt,
     return sq::linear_layout(M, N, K, in_dt, out_dt).total;
 }
 
+sq_status sq_linear_workspace_offsets(int64_t M, int64_t N, int64_t K, sq_dtype in_dt, sq_dtype out_dt,
+                                      size_t* offsets) {
+    if (M < 0 || N < 0 || K < 0 || !offsets) {
+        sq::set_error("negative size or NULL offsets");
+        return SQ_ERR_INVALID_ARG;
+    }
+    if ((in_dt != SQ_F32 && in_dt != SQ_BF16) || (out_dt != SQ_F32 && out_dt != SQ_BF16)) {
+        sq::set_error("input and output dtypes must be SQ_F32 or SQ_BF16");
+        return SQ_ERR_UNSUPPORTED;
+    }
+    const sq::LinearLayout L = sq::linear_layout(M, N, K, in_dt, out_dt);
+    offsets[0] = L.xmax;
+    offsets[1] = L.wmax;
+    offsets[2] = L.s;
+    offsets[3] = L.xq;
+    offsets[4] = L.xs;
+    offsets[5] = L.wq;
+    offsets[6] = L.wsc;
+    return SQ_OK;
+}
+
 sq_status sq_linear(const void* x, const void* w, sq_dtype in_dt, int64_t M, int64_t N, int64_t K,
                     float alpha, float eps, void* y, sq_dtype out_dt, void* workspace, size_t ws_bytes,
                     sq_stream_t stream) {

@@ -27,6 +27,22 @@ __device__ __forceinline__ void record_status(unsigned int code, unsigned int si
     if (atomicCAS(&g_status, 0u, code) == 0u) atomicExch(&g_status_site, site);
 }
 
+// ---------------------------------------------------------------- debug index checks
+// A build with -DSQ_DEBUG checks, before the global stores whose indices the
+// kernels do not otherwise guard (rows that fill every lane, rare-path
+// repairs, vector stores, cluster ranks), that the access is inside its
+// buffer; a failed check records SQ_ERR_BOUNDS with the store's site in the
+// status word (sq_get_status reports it) and the store is skipped. Nothing
+// traps. Without SQ_DEBUG every check is the constant true.
+#ifdef SQ_DEBUG
+__device__ __forceinline__ bool dchk(bool ok, unsigned int site) {
+    if (!ok) record_status(SQ_ERR_BOUNDS, site);
+    return ok;
+}
+#else
+__device__ __forceinline__ bool dchk(bool, unsigned int) { return true; }
+#endif
+
 // ---------------------------------------------------------------- bf16 / misc
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
@@ -182,6 +198,16 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t
                  : "memory");
 }
 
+// The same for bf16: kind::f16 with bf16 A and B, fp32 D.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -219,6 +245,16 @@ __host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N) {
     return (1u << 4)                          // D format: f32
          | (0u << 7)                          // A format: E4M3
          | (0u << 10)                         // B format: E4M3
+         | ((uint32_t)(N >> 3) << 17)         // N / 8
+         | ((uint32_t)(M >> 4) << 24);        // M / 16
+}
+
+// Instruction descriptor, kind::f16 with bf16 A and B (format code 1) and fp32
+// D (format code 1), both operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N) {
+    return (1u << 4)                          // D format: f32
+         | (1u << 7)                          // A format: bf16
+         | (1u << 10)                         // B format: bf16
          | ((uint32_t)(N >> 3) << 17)         // N / 8
          | ((uint32_t)(M >> 4) << 24);        // M / 16
 }

@@ -50,6 +50,14 @@ constexpr int TMEM_COLS = 2 * ACC_COLS;         // double-buffered: 512 columns
 constexpr int GEMM_THREADS = 192;               // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint32_t IDESC_TILED = make_idesc_i8(BM, BN);
 constexpr uint32_t IDESC_TILED_E4M3 = make_idesc_e4m3(BM, BN);
+constexpr uint32_t IDESC_TILED_BF16 = make_idesc_bf16(BM, BN);
+
+// Operand kinds of the 1-CTA kernel: int8 codes (the layer's GEMM), FP8 E4M3
+// codes, or bf16 values (the plain floating-point product of the alpha
+// search, fp32 accumulation, raw fp32 output).
+enum OperandKind { kAkI8 = 0, kAkE4M3 = 1, kAkBF16 = 2 };
+// Elements of one 128-byte k-block row.
+__host__ __device__ constexpr int bk_elems(int ak) { return ak == kAkBF16 ? 64 : 128; }
 
 constexpr int S_BM = 128;        // weight rows per tile (MMA M)
 constexpr int S_BN = 16;         // tokens (MMA N)
@@ -71,10 +79,11 @@ constexpr size_t stream_smem_bytes() {
     return 1024 + S_STAGES * (S_A_STAGE + S_B_STAGE) + 256;
 }
 
-// One MMA of the 1-CTA kernel: int8 or FP8 E4M3 operands.
-template <bool F8>
+// One MMA of the 1-CTA kernel (32 bytes of K): int8, FP8 E4M3 or bf16 operands.
+template <int AK>
 __device__ __forceinline__ void mma_tiled(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
-    if (F8) mma_f8(d_tmem, adesc, bdesc, IDESC_TILED_E4M3, accumulate);
+    if (AK == kAkE4M3) mma_f8(d_tmem, adesc, bdesc, IDESC_TILED_E4M3, accumulate);
+    else if (AK == kAkBF16) mma_bf16(d_tmem, adesc, bdesc, IDESC_TILED_BF16, accumulate);
     else mma_i8(d_tmem, adesc, bdesc, IDESC_TILED, accumulate);
 }
 
@@ -167,8 +176,9 @@ __device__ __forceinline__ float add_split1(float v, int64_t t, int64_t n, const
     return v;
 }
 
-// Stores 32 consecutive outputs of one row (row-major y, row stride N).
-template <int OUT, bool SPLIT, bool F8 = false>
+// Stores 32 consecutive outputs of one row (row-major y, row stride N). For
+// bf16 operands (AK == kAkBF16) the outputs are the raw fp32 accumulators.
+template <int OUT, bool SPLIT, int AK = kAkI8>
 __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int N, const uint32_t (&r)[32],
                                             float sa, const float* __restrict__ w_scale, const float* xr,
                                             const float* ws_col, int ld) {
@@ -186,8 +196,12 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
         }
         return;
     }
+    constexpr bool F8 = AK == kAkE4M3;
     float v[32];
-    if (full) {
+    if (AK == kAkBF16) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    } else if (full) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
             const float4 sw = __ldg(reinterpret_cast<const float4*>(w_scale + col0 + i));
@@ -207,7 +221,8 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
         if (full && (N & 3) == 0) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(yp + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                if (dchk((reinterpret_cast<uintptr_t>(yp + i) & 15u) == 0, SITE_DBG_GEMM_VECTOR))
+                    *reinterpret_cast<float4*>(yp + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
         } else {
             for (int i = 0; i < 32; ++i)
                 if (col0 + i < N) yp[i] = v[i];
@@ -222,7 +237,8 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
                 pk.y = pack_bf16x2(v[i + 2], v[i + 3]);
                 pk.z = pack_bf16x2(v[i + 4], v[i + 5]);
                 pk.w = pack_bf16x2(v[i + 6], v[i + 7]);
-                *reinterpret_cast<uint4*>(yp + i) = pk;
+                if (dchk((reinterpret_cast<uintptr_t>(yp + i) & 15u) == 0, SITE_DBG_GEMM_VECTOR))
+                    *reinterpret_cast<uint4*>(yp + i) = pk;
             }
         } else {
             for (int i = 0; i < 32; ++i)
@@ -232,7 +248,7 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
 }
 
 // ================================================================== prefill
-template <int OUT, bool SPLIT, bool F8 = false>
+template <int OUT, bool SPLIT, int AK = kAkI8>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const float* __restrict__ x_scale, const float* __restrict__ w_scale,
@@ -250,7 +266,8 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
     const int num_tiles = num_m * num_n;
-    const int num_kb = (K + BK - 1) / BK;
+    constexpr int BKE = bk_elems(AK);   // elements per k-block
+    const int num_kb = (K + BKE - 1) / BKE;
 
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const int FULL = 0, EMPTY = STAGES, TFULL = 2 * STAGES, TEMPTY = 2 * STAGES + 2, DRAIN = 2 * STAGES + 4;
@@ -305,8 +322,8 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                         break;
                     }
                     mbar_arrive_expect_tx(bar(FULL + stage), A_STAGE + B_STAGE);
-                    tma_load_2d(smem_u32(sA + stage * A_STAGE), &tmA, bar(FULL + stage), kb * BK, mb * BM);
-                    tma_load_2d(smem_u32(sB + stage * B_STAGE), &tmB, bar(FULL + stage), kb * BK, nb * BN);
+                    tma_load_2d(smem_u32(sA + stage * A_STAGE), &tmA, bar(FULL + stage), kb * BKE, mb * BM);
+                    tma_load_2d(smem_u32(sB + stage * B_STAGE), &tmB, bar(FULL + stage), kb * BKE, nb * BN);
                     ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -342,7 +359,7 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k)
-                        mma_tiled<F8>(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
+                        mma_tiled<AK>(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
                                make_sw128_kmajor_desc(b0 + k * UMMA_K),
                                (kb | k) != 0 ? 1u : 0u);
                     mma_commit(bar(EMPTY + stage));
@@ -373,7 +390,7 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             tc_fence_after();
             const int64_t row = (int64_t)mb * BM + quarter * 32 + lane;
             const bool row_ok = row < M;
-            const float sa = (OUT != kOutI32 && row_ok) ? __ldg(x_scale + row) : 0.0f;
+            const float sa = (OUT != kOutI32 && AK != kAkBF16 && row_ok) ? __ldg(x_scale + row) : 0.0f;
             const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; c += 2) {
@@ -384,9 +401,9 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 const int col0 = nb * BN + c * 32;
                 const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
                 if (row_ok && col0 < N)
-                    store_row32<OUT, SPLIT, F8>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
+                    store_row32<OUT, SPLIT, AK>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
                 if (row_ok && col0 + 32 < N)
-                    store_row32<OUT, SPLIT, F8>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
+                    store_row32<OUT, SPLIT, AK>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
             }
             tc_fence_before();
             __syncwarp();
@@ -659,9 +676,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const int col0 = nb * BN + c * 32;
                 const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
                 if (row_ok && col0 < N)
-                    store_row32<OUT, SPLIT, F8>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
+                    store_row32<OUT, SPLIT, F8 ? kAkE4M3 : kAkI8>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
                 if (row_ok && col0 + 32 < N)
-                    store_row32<OUT, SPLIT, F8>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
+                    store_row32<OUT, SPLIT, F8 ? kAkE4M3 : kAkI8>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
             }
             tc_fence_before();
             __syncwarp();
@@ -893,6 +910,302 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     }
 }
 
+// ================================================================== decode, clusters
+// The same swap-AB product (weight rows on the MMA's 128-row side, the tokens
+// as N = 16), with the split-K partial sums merged inside thread-block
+// clusters instead of through global memory.
+//
+// Work split: the 128-row weight tiles are dealt to the clusters in contiguous
+// runs of whole tiles; inside a cluster, the (tile, k-block) units of its tiles
+// are split evenly between its CTAs in contiguous ranges. A CTA accumulates
+// each run of its units inside one tile (a segment) in TMEM. The CTA holding a
+// tile's first k-block owns the tile and writes its rows of Y. Every other CTA
+// holding units of that tile -- for a given CTA this can only be its first
+// segment, and an owner can receive only into its last segment -- adds its
+// partial sums into the owner's receive buffer in shared memory with
+// distributed-shared-memory integer atomics (exact and order-free) and then
+// arrives, with release semantics at cluster scope, on the owner's receive
+// barrier. The owner's epilogue waits (bounded, acquire at cluster scope) for
+// the arrivals it expects, adds the buffer to its own TMEM partial sums and
+// applies the epilogue. Nothing is written to global memory but Y.
+//
+// Segment bookkeeping is pure arithmetic on the static split, identical in
+// every CTA of the cluster.
+struct DecodeSplit {
+    int rank, csize;          // this CTA's rank in the cluster, the cluster size
+    long long units;          // units of the cluster's tiles
+    int tile0;                // the cluster's first tile
+    int num_kb;
+    __device__ long long begin(int r) const { return units * r / csize; }
+    // rank holding local unit u (u < units)
+    __device__ int holder(long long u) const {
+        int r = (int)((u * csize) / units);
+        while (r + 1 < csize && begin(r + 1) <= u) ++r;
+        while (r > 0 && begin(r) > u) --r;
+        return r;
+    }
+};
+
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t local_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void red_add_cluster(uint32_t cluster_addr, int32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.add.s32 [%0], %1;" :: "r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void arrive_remote_release(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_acq_cluster(uint32_t bar, uint32_t parity, long long limit,
+                                                      volatile int* abort, unsigned int site) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit) {
+            *abort = 1;
+            record_status(SQ_ERR_TIMEOUT, site);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+constexpr size_t DC_RECV_BYTES = (size_t)S_BN * S_BM * sizeof(int32_t);   // 8 KB: [token][row] int32
+constexpr size_t decode_cluster_smem_bytes() {
+    return 1024 + S_STAGES * (S_A_STAGE + S_B_STAGE) + DC_RECV_BYTES + 256;
+}
+
+template <int OUT>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_decode_cluster_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                           const float* __restrict__ x_scale, const float* __restrict__ w_scale,
+                           void* __restrict__ y, int M, int N, int K, long long wait_limit) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + S_STAGES * S_A_STAGE;
+    int32_t* recv = reinterpret_cast<int32_t*>(sB + S_STAGES * S_B_STAGE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(recv) + DC_RECV_BYTES);
+    // bars: full[S_STAGES] | empty[S_STAGES] | tfull[2] | tempty[2] | drain | recv
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * S_STAGES + 6);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    __shared__ int no_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = (N + S_BM - 1) / S_BM;
+    const int num_kb = (K + BK - 1) / BK;
+    DecodeSplit sp;
+    sp.csize = (int)cluster_nctarank();
+    sp.rank = (int)cluster_rank();
+    const int cl = blockIdx.x / sp.csize, ncl = gridDim.x / sp.csize;
+    sp.tile0 = (int)((long long)num_tiles * cl / ncl);
+    const int tile1 = (int)((long long)num_tiles * (cl + 1) / ncl);
+    sp.num_kb = num_kb;
+    sp.units = (long long)(tile1 - sp.tile0) * num_kb;
+    const long long u_begin = sp.begin(sp.rank), u_end = sp.begin(sp.rank + 1);
+
+    auto bar = [&](int i) { return smem_u32(bars + i); };
+    const int FULL = 0, EMPTY = S_STAGES, TFULL = 2 * S_STAGES, TEMPTY = 2 * S_STAGES + 2, DRAIN = 2 * S_STAGES + 4,
+              RECV = 2 * S_STAGES + 5;
+
+    // Contributors to this CTA's last segment (if it is owned and the tile
+    // continues past this CTA's range): the CTAs holding the rest of the tile.
+    int n_contrib = 0;
+    if (u_end > u_begin) {
+        const long long last_lo = max(u_begin, ((u_end - 1) / num_kb) * num_kb);
+        const long long tile_end = ((u_end - 1) / num_kb + 1) * num_kb;
+        if (last_lo % num_kb == 0 && u_end < tile_end) {
+            const int last = sp.holder(tile_end - 1);
+            for (int q = sp.rank + 1; q <= last; ++q) n_contrib += sp.begin(q) < sp.begin(q + 1) ? 1 : 0;
+        }
+    }
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S_STAGES; ++s) {
+            mbar_init(bar(FULL + s), 1);
+            mbar_init(bar(EMPTY + s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar(TFULL + a), 1);
+            mbar_init(bar(TEMPTY + a), 4);
+        }
+        mbar_init(bar(DRAIN), 1);
+        mbar_init(bar(RECV), n_contrib > 0 ? (uint32_t)(128 * n_contrib) : 1u);
+        *abort_flag = 0;
+        no_abort = 0;
+        fence_barrier_init();
+    }
+    for (int i = threadIdx.x; i < (int)(DC_RECV_BYTES / 16); i += GEMM_THREADS)
+        reinterpret_cast<uint4*>(recv)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc<S_TMEM_COLS>(smem_u32(tmem_holder));
+        tc_fence_before();
+    }
+    // every CTA's barriers and receive buffer are ready before any remote access
+    __syncwarp();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (long long u = u_begin; u < u_end && ok; ++u) {
+                const int tile = sp.tile0 + (int)(u / num_kb), kb = (int)(u % num_kb);
+                if (!mbar_wait(bar(EMPTY + stage), phase ^ 1, wait_limit, abort_flag, SITE_STREAM_PRODUCER)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(bar(FULL + stage), S_A_STAGE + S_B_STAGE);
+                tma_load_2d(smem_u32(sA + stage * S_A_STAGE), &tmW, bar(FULL + stage), kb * BK, tile * S_BM);
+                tma_load_2d(smem_u32(sB + stage * S_B_STAGE), &tmX, bar(FULL + stage), kb * BK, 0);
+                ++issued;
+                if (++stage == S_STAGES) { stage = 0; phase ^= 1; }
+            }
+            if (!ok || *abort_flag) {
+                for (int s = 0; s < S_STAGES; ++s) {
+                    const long long cnt = issued / S_STAGES + (s < issued % S_STAGES ? 1 : 0);
+                    if (cnt > 0)
+                        mbar_wait(bar(FULL + s), (uint32_t)((cnt - 1) & 1), wait_limit, &no_abort, SITE_STREAM_DRAIN);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            long long u = u_begin;
+            while (u < u_end && ok) {
+                const long long seg_end = min(u_end, (u / num_kb + 1) * num_kb);
+                if (!mbar_wait(bar(TEMPTY + acc), acc_phase ^ 1, wait_limit, abort_flag, SITE_STREAM_MMA_TMEM)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S_BN);
+                bool first = true;
+                for (; u < seg_end; ++u) {
+                    if (!mbar_wait(bar(FULL + stage), phase, wait_limit, abort_flag, SITE_STREAM_MMA_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * S_A_STAGE);
+                    const uint32_t b0 = smem_u32(sB + stage * S_B_STAGE);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k)
+                        mma_i8(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
+                               make_sw128_kmajor_desc(b0 + k * UMMA_K), IDESC_STREAM, (first && k == 0) ? 0u : 1u);
+                    first = false;
+                    mma_commit(bar(EMPTY + stage));
+                    if (++stage == S_STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(bar(TFULL + acc));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            mma_commit(bar(DRAIN));
+            mbar_wait(bar(DRAIN), 0, wait_limit, &no_abort, SITE_STREAM_DRAIN);
+        }
+        __syncwarp();
+    } else {
+        // Epilogue: warp `quarter` owns weight rows quarter*32 .. +32 of each
+        // tile (its TMEM lane quarter); lane l holds row quarter*32 + l.
+        const int quarter = warp & 3;
+        const int row_in_tile = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        long long u = u_begin;
+        while (u < u_end) {
+            const long long seg_lo = u;
+            const long long seg_hi = min(u_end, (u / num_kb + 1) * num_kb);
+            const int tile = sp.tile0 + (int)(seg_lo / num_kb);
+            u = seg_hi;
+            if (!mbar_wait(bar(TFULL + acc), acc_phase, wait_limit, abort_flag, SITE_STREAM_EPILOGUE)) break;
+            tc_fence_after();
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * S_BN), r);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(TEMPTY + acc));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+
+            if (seg_lo % num_kb != 0) {
+                // a contribution to the tile's owner
+                const int owner = sp.holder((seg_lo / num_kb) * num_kb);
+                // the owner holds the tile's first unit, before this CTA's range
+                if (!dchk(owner >= 0 && owner < sp.rank, SITE_DBG_DECODE_OWNER)) continue;
+                const uint32_t rbase = mapa_rank(smem_u32(recv), (uint32_t)owner);
+#pragma unroll
+                for (int t = 0; t < S_BN; ++t)
+                    if (t < M) red_add_cluster(rbase + (uint32_t)((t * S_BM + row_in_tile) * 4), (int32_t)r[t]);
+                arrive_remote_release(mapa_rank(bar(RECV), (uint32_t)owner));
+                continue;
+            }
+            if (seg_hi % num_kb != 0 && n_contrib > 0) {
+                // owned, and the rest of the tile comes from the next CTAs
+                if (!mbar_wait_acq_cluster(bar(RECV), 0, wait_limit, abort_flag, SITE_STREAM_EPILOGUE)) break;
+#pragma unroll
+                for (int t = 0; t < S_BN; ++t)
+                    if (t < M) r[t] = (uint32_t)((int32_t)r[t] + recv[t * S_BM + row_in_tile]);
+            }
+            const int n = tile * S_BM + row_in_tile;
+            if (n < N) {
+                const float sw = (OUT != kOutI32) ? __ldg(w_scale + n) : 0.0f;
+#pragma unroll
+                for (int t = 0; t < S_BN; ++t) {
+                    if (t < M) {
+                        const int64_t o = (int64_t)t * N + n;
+                        if (OUT == kOutI32) {
+                            static_cast<int32_t*>(y)[o] = (int32_t)r[t];
+                        } else {
+                            const float v = dequant((int32_t)r[t], __ldg(x_scale + t), sw);
+                            if (OUT == kOutF32) static_cast<float*>(y)[o] = v;
+                            else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // no CTA leaves while another may still add into its shared memory
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc<S_TMEM_COLS>(tmem_base);
+    }
+}
+
 // ================================================================== host side
 namespace {
 
@@ -934,6 +1247,26 @@ sq_status make_map_i8(CUtensorMap* map, const void* base, int64_t rows, int64_t 
     return SQ_OK;
 }
 
+// Row-major bf16 matrix [rows x K] as a 2-D tensor map with 128B swizzle and a
+// (64 elements = 128 bytes of K) x box_rows box.
+sq_status make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
+    sq_status r = get_encoder();
+    if (r != SQ_OK) return r;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64u, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult cr = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d) for a %lld x %lld bf16 matrix", (int)cr,
+                  (long long)rows, (long long)K);
+        return SQ_ERR_CUDA;
+    }
+    return SQ_OK;
+}
+
 template <typename Kern>
 sq_status ensure_smem_attr(Kern k, size_t bytes, bool& done) {
     // Per device: the attribute is a property of the function on the current device.
@@ -946,17 +1279,17 @@ sq_status ensure_smem_attr(Kern k, size_t bytes, bool& done) {
     return SQ_OK;
 }
 
-template <int OUT, bool SPLIT = false, bool F8 = false>
+template <int OUT, bool SPLIT = false, int AK = kAkI8>
 sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
                        int M, int N, int K, cudaStream_t st, const SplitTerm& sp = SplitTerm{}) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const size_t smem = tiled_smem_bytes() + (SPLIT ? kSplitSmem : 0);
-    sq_status r = ensure_smem_attr(gemm_tiled_kernel<OUT, SPLIT, F8>, smem, attr_done[di.device & 63]);
+    sq_status r = ensure_smem_attr(gemm_tiled_kernel<OUT, SPLIT, AK>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = tiles < di.sm_count ? tiles : di.sm_count;
-    return launch_pdl("gemm_tiled_kernel", gemm_tiled_kernel<OUT, SPLIT, F8>, dim3(grid), dim3(GEMM_THREADS), smem, st, 1,
+    return launch_pdl("gemm_tiled_kernel", gemm_tiled_kernel<OUT, SPLIT, AK>, dim3(grid), dim3(GEMM_THREADS), smem, st, 1,
                       ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
 }
 
@@ -988,6 +1321,87 @@ sq_status launch_stream(const CUtensorMap& tw, const CUtensorMap& tx, const floa
     const int grid = units < di.sm_count ? (int)units : di.sm_count;
     return launch_pdl("gemm_stream_kernel", gemm_stream_kernel<OUT, SPLIT>, dim3(grid), dim3(GEMM_THREADS), smem, st,
                       1, tw, tx, xs, wsc, y, M, N, K, ws_acc, counts, sp, wait_limit_cycles());
+}
+
+// Cluster sizes the decode kernel may use, and how many clusters of each can
+// be resident at once on the current device (queried once per device).
+constexpr int kDecodeClusterSizes[4] = {2, 4, 8, 16};
+
+struct DecodeClusterInfo {
+    bool ready = false;
+    int max_clusters[4] = {0, 0, 0, 0};
+};
+DecodeClusterInfo g_dc_info[64];
+std::mutex g_dc_mu;
+
+sq_status decode_cluster_info(DecodeClusterInfo& out) {
+    const DeviceInfo& di = device_info();
+    std::lock_guard<std::mutex> lk(g_dc_mu);
+    DecodeClusterInfo& d = g_dc_info[di.device & 63];
+    if (!d.ready) {
+        const size_t smem = decode_cluster_smem_bytes();
+        auto kern = gemm_decode_cluster_kernel<kOutBF16>;
+        cudaError_t e;
+        const void* fns[3] = {(const void*)gemm_decode_cluster_kernel<kOutF32>,
+                              (const void*)gemm_decode_cluster_kernel<kOutBF16>,
+                              (const void*)gemm_decode_cluster_kernel<kOutI32>};
+        for (const void* f : fns) {
+            if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+                return cuda_fail(e, "cudaFuncSetAttribute(max dynamic shared memory)");
+            if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
+                return cuda_fail(e, "cudaFuncSetAttribute(non-portable cluster size)");
+        }
+        for (int i = 0; i < 4; ++i) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(kDecodeClusterSizes[i] * 8);
+            cfg.blockDim = dim3(GEMM_THREADS);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr;
+            attr.id = cudaLaunchAttributeClusterDimension;
+            attr.val.clusterDim.x = kDecodeClusterSizes[i];
+            attr.val.clusterDim.y = 1;
+            attr.val.clusterDim.z = 1;
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                n = 0;
+            }
+            d.max_clusters[i] = n;
+        }
+        d.ready = true;
+    }
+    out = d;
+    return SQ_OK;
+}
+
+// The cluster size with the fewest units on the busiest CTA (ties: the
+// smaller size); 0 if no cluster size can be launched.
+int pick_decode_cluster(const DecodeClusterInfo& info, int num_tiles, int num_kb, int& ncl_out) {
+    long long best = -1;
+    int best_c = 0;
+    for (int i = 0; i < 4; ++i) {
+        const int c = kDecodeClusterSizes[i];
+        const int ncl = std::min(info.max_clusters[i], num_tiles);
+        if (ncl <= 0) continue;
+        const long long tiles = (num_tiles + ncl - 1) / ncl;
+        const long long busiest = (tiles * num_kb + c - 1) / c;
+        if (best < 0 || busiest < best) {
+            best = busiest;
+            best_c = c;
+            ncl_out = ncl;
+        }
+    }
+    return best_c;
+}
+
+template <int OUT>
+sq_status launch_decode_cluster(const CUtensorMap& tw, const CUtensorMap& tx, const float* xs, const float* wsc,
+                                void* y, int M, int N, int K, int csize, int ncl, cudaStream_t st) {
+    return launch_pdl("gemm_decode_cluster_kernel", gemm_decode_cluster_kernel<OUT>, dim3(csize * ncl),
+                      dim3(GEMM_THREADS), decode_cluster_smem_bytes(), st, (unsigned)csize, tw, tx, xs, wsc, y, M, N,
+                      K, wait_limit_cycles());
 }
 
 size_t stream_ws_bytes(int64_t M, int64_t N) {
@@ -1040,6 +1454,21 @@ sq_status gemm_dispatch(const int8_t* xq, const float* x_scale, const int8_t* wq
         CUtensorMap tw, tx;
         if ((r = make_map_i8(&tw, wq, N, K, S_BM)) != SQ_OK) return r;
         if ((r = make_map_i8(&tx, xq, M, K, S_BN)) != SQ_OK) return r;
+        if (!sp_on) {
+            // the cluster kernel merges its partial sums on chip and needs no
+            // workspace; the workspace serves the decomposed path's kernel
+            DecodeClusterInfo info;
+            if ((r = decode_cluster_info(info)) != SQ_OK) return r;
+            int ncl = 0;
+            const int csize = pick_decode_cluster(info, (int)((N + S_BM - 1) / S_BM), (int)((K + BK - 1) / BK), ncl);
+            if (csize > 0) {
+                switch (out) {
+                    case kOutF32: return launch_decode_cluster<kOutF32>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, csize, ncl, st);
+                    case kOutBF16: return launch_decode_cluster<kOutBF16>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, csize, ncl, st);
+                    default: return launch_decode_cluster<kOutI32>(tw, tx, x_scale, w_scale, y, (int)M, (int)N, (int)K, csize, ncl, st);
+                }
+            }
+        }
         int32_t* ws_acc = static_cast<int32_t*>(workspace);
         const size_t acc_al = (((size_t)M * N * 4) + 255) & ~size_t(255);
         unsigned int* counts = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + acc_al);
@@ -1109,8 +1538,75 @@ sq_status gemm_e4m3_impl(const uint8_t* xq, const float* x_scale, const uint8_t*
     if ((r = make_map_i8(&ta, xq, M, K, BM)) != SQ_OK) return r;
     if ((r = make_map_i8(&tb, wq, N, K, BN)) != SQ_OK) return r;
     return out_dt == SQ_F32
-        ? launch_tiled<kOutF32, false, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, none)
-        : launch_tiled<kOutBF16, false, true>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, none);
+        ? launch_tiled<kOutF32, false, kAkE4M3>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, none)
+        : launch_tiled<kOutBF16, false, kAkE4M3>(ta, tb, x_scale, w_scale, y, (int)M, (int)N, (int)K, st, none);
+}
+
+// ------------------------------------------------------------------ plain floating-point products
+// y [M x N] fp32 = x [M x K] . w [N x K]^T, the reference product of the alpha
+// search. bf16 operands: the 1-CTA tcgen05 kernel with kind::f16 (every
+// product exact in fp32, the sum accumulated in fp32 in TMEM, its order the
+// tensor core's). fp32 operands: a CUDA-core kernel, each output a chain of
+// fp32 fused multiply-adds in k order.
+constexpr int SG_TM = 64, SG_TN = 64, SG_TK = 16, SG_THREADS = 256;
+
+__global__ void __launch_bounds__(SG_THREADS)
+sgemm_xwt_kernel(const float* __restrict__ x, const float* __restrict__ w, float* __restrict__ y, int M, int N,
+                 int K) {
+    __shared__ float xs[SG_TK][SG_TM + 4];
+    __shared__ float ws[SG_TK][SG_TN + 4];
+    pdl_wait();
+    pdl_trigger();
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;   // 16 x 16 threads, 4 x 4 outputs each
+    const int m0 = blockIdx.y * SG_TM, n0 = blockIdx.x * SG_TN;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < K; k0 += SG_TK) {
+        for (int i = threadIdx.x; i < SG_TM * SG_TK; i += SG_THREADS) {
+            const int r = i / SG_TK, c = i % SG_TK;
+            const int gm = m0 + r, gn = n0 + r, gk = k0 + c;
+            xs[c][r] = (gm < M && gk < K) ? __ldg(x + (int64_t)gm * K + gk) : 0.0f;
+            ws[c][r] = (gn < N && gk < K) ? __ldg(w + (int64_t)gn * K + gk) : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < SG_TK; ++c) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[i] = xs[c][ty * 4 + i];
+                b[i] = ws[c][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
+            if (gm < M && gn < N) y[(int64_t)gm * N + gn] = acc[i][j];
+        }
+}
+
+sq_status float_gemm_xwt(const void* x, const void* w, sq_dtype dt, int64_t M, int64_t N, int64_t K, float* y,
+                         cudaStream_t st) {
+    if (M <= 0 || N <= 0) return SQ_OK;
+    if (M > 2147483647LL || N > 2147483647LL || K > 2147483647LL) { set_error("size too large"); return SQ_ERR_UNSUPPORTED; }
+    if (dt == SQ_BF16) {
+        if (K % 8 != 0) { set_error("K must be a multiple of 8 for bf16 operands"); return SQ_ERR_UNSUPPORTED; }
+        CUtensorMap ta, tb;
+        sq_status r;
+        if ((r = make_map_bf16(&ta, x, M, K, BM)) != SQ_OK) return r;
+        if ((r = make_map_bf16(&tb, w, N, K, BN)) != SQ_OK) return r;
+        return launch_tiled<kOutF32, false, kAkBF16>(ta, tb, nullptr, nullptr, y, (int)M, (int)N, (int)K, st);
+    }
+    const dim3 grid((unsigned)((N + SG_TN - 1) / SG_TN), (unsigned)((M + SG_TM - 1) / SG_TM));
+    return launch_pdl("sgemm_xwt_kernel", sgemm_xwt_kernel, grid, dim3(SG_THREADS), 0, st, 1,
+                      static_cast<const float*>(x), static_cast<const float*>(w), y, (int)M, (int)N, (int)K);
 }
 
 sq_status gemm_split_impl(const int8_t* xq, const float* x_scale, const int8_t* wq, const float* w_scale,

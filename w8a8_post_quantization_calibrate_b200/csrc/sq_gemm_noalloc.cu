@@ -23,7 +23,8 @@ namespace sq {
 namespace {
 
 // Maximum scratch: M*N int32 partial sums (at most 1 MiB, so M*N <= 262,144)
-// plus 4 counters per 128-row weight tile (at most 32 KiB, so N <= 262,144).
+// plus 4 counters per 128-row weight tile (32 KiB would take N up to 262,144;
+// since M >= 1, the M*N limit already keeps N, and so the counters, within it).
 constexpr size_t kNoallocAccBytes = size_t(1) << 20;
 constexpr size_t kNoallocCountBytes = size_t(32) << 10;
 constexpr size_t kNoallocScratchBytes = kNoallocAccBytes + kNoallocCountBytes;
@@ -76,10 +77,10 @@ sq_status gemm_noalloc(const int8_t* xq, const float* x_scale, const int8_t* wq,
         set_error("sq_w8a8_gemm_noalloc: M=%lld exceeds its maximum of %d", (long long)M, STREAM_MAX_M);
         return SQ_ERR_UNSUPPORTED;
     }
+    // The N test is a guard only: M >= 1 and the M*N limit already bound N.
     if (M * N > (int64_t)(kNoallocAccBytes / sizeof(int32_t)) || N > (int64_t)(kNoallocCountBytes / 16) * S_BM) {
-        set_error("sq_w8a8_gemm_noalloc: M*N=%lld (N=%lld) exceeds its scratch (M*N <= %zu, N <= %zu)",
-                  (long long)(M * N), (long long)N, kNoallocAccBytes / sizeof(int32_t),
-                  (kNoallocCountBytes / 16) * S_BM);
+        set_error("sq_w8a8_gemm_noalloc: M*N=%lld exceeds its scratch (M*N <= %zu)", (long long)(M * N),
+                  kNoallocAccBytes / sizeof(int32_t));
         return SQ_ERR_UNSUPPORTED;
     }
     if (K == 0 || K % 16 != 0) { set_error("K=%lld must be a positive multiple of 16", (long long)K); return SQ_ERR_UNSUPPORTED; }
@@ -112,7 +113,21 @@ sq_status gemm_noalloc(const int8_t* xq, const float* x_scale, const int8_t* wq,
     }
 }
 
+// Test hook: overwrite the whole scratch array with a non-zero byte pattern,
+// as a call that stopped early would leave it.
+sq_status noalloc_dirty(cudaStream_t st) {
+    unsigned char* scratch = nullptr;
+    sq_status r = noalloc_scratch(&scratch);
+    if (r != SQ_OK) return r;
+    cudaError_t e = cudaMemsetAsync(scratch, 0xA5, kNoallocScratchBytes, st);
+    return e == cudaSuccess ? SQ_OK : cuda_fail(e, "dirty no-alloc scratch");
+}
+
 }  // namespace sq
+
+extern "C" sq_status sq_selftest_dirty_noalloc_scratch(sq_stream_t stream) {
+    return sq::noalloc_dirty((cudaStream_t)stream);
+}
 
 extern "C" sq_status sq_w8a8_gemm_noalloc(const int8_t* xq, const float* x_scale, const int8_t* wq,
                                           const float* w_scale, int64_t M, int64_t N, int64_t K, void* y,

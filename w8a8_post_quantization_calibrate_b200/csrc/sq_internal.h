@@ -81,6 +81,12 @@ enum Site : unsigned int {
     SITE_STREAM_DRAIN = 24,
     SITE_QUANT_WAIT = 30,
     SITE_QUANT_DRAIN = 31,
+    SITE_PROBE = 40,
+    SITE_DBG_RING_CODES = 50,
+    SITE_DBG_RING_REPAIR = 51,
+    SITE_DBG_RING_SCALE = 52,
+    SITE_DBG_GEMM_VECTOR = 53,
+    SITE_DBG_DECODE_OWNER = 54,
 };
 
 // Internal entry points used by sq_linear.

@@ -5,6 +5,7 @@
 #include "sq_quant.cu"
 #include "sq_act_variants.cu"
 #include "sq_gemm.cu"
+#include "sq_probe.cu"
 #include "sq_split.cu"
 #include "sq_gemm_noalloc.cu"
 #include "sq_search.cu"

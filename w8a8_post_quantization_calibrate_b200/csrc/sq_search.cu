@@ -6,8 +6,10 @@
 // Explained", "Alpha: how much difficulty to move": alpha is a per-model
 // tuning parameter).
 //
-// Y is a plain floating-point GEMM, computed once by cuBLAS (bf16 or fp32
-// operands, fp32 accumulation). Each candidate then costs a2, a3, a4, the int8
+// Y is a plain floating-point GEMM computed once by this library's kernels:
+// for bf16 operands the tcgen05 GEMM with kind::f16 (exact products, fp32
+// accumulation in TMEM), for fp32 operands a CUDA-core kernel (fp32 fused
+// multiply-adds in k order). Each candidate then costs a2, a3, a4, the int8
 // GEMM with fp32 output and one error reduction: a grid-strided pass that
 // accumulates sum (Yq - Y)^2 and sum Y^2 in fp64 per block, and a one-block
 // pass that adds the block sums in a fixed order (deterministic on a given
@@ -15,7 +17,6 @@
 #include <cmath>
 #include <mutex>
 
-#include <cublas_v2.h>
 #include <cuda_runtime.h>
 
 #include "sq_device.cuh"
@@ -132,41 +133,10 @@ SearchLayout search_layout(int64_t T, int64_t N, int64_t K, int64_t n_alpha) {
     return L;
 }
 
-std::mutex g_blas_mu;
-cublasHandle_t g_blas[64] = {};
-
-sq_status blas_handle(cublasHandle_t& h) {
-    const int dev = device_info().device;
-    std::lock_guard<std::mutex> lock(g_blas_mu);
-    if (!g_blas[dev & 63]) {
-        if (cublasCreate(&g_blas[dev & 63]) != CUBLAS_STATUS_SUCCESS) {
-            set_error("cublasCreate failed");
-            return SQ_ERR_CUDA;
-        }
-    }
-    h = g_blas[dev & 63];
-    return SQ_OK;
-}
-
-// yref [T x N] row-major = X W^T: in cuBLAS's column-major terms,
-// yref^T [N x T] = W [N x K] . X^T, i.e. op(A) = W (A = W viewed as K x N, transposed)
-// and op(B) = X^T (B = X viewed as K x T).
+// yref [T x N] row-major = X W^T, by this library's own kernels.
 sq_status reference_gemm(const void* x, const void* w, sq_dtype dt, int64_t T, int64_t N, int64_t K, float* yref,
                          cudaStream_t st) {
-    cublasHandle_t h;
-    sq_status r = blas_handle(h);
-    if (r != SQ_OK) return r;
-    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) { set_error("cublasSetStream failed"); return SQ_ERR_CUDA; }
-    const float one = 1.0f, zero = 0.0f;
-    const cudaDataType_t in = dt == SQ_F32 ? CUDA_R_32F : CUDA_R_16BF;
-    const cublasStatus_t s = cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, (int)N, (int)T, (int)K, &one, w, in, (int)K,
-                                          x, in, (int)K, &zero, yref, CUDA_R_32F, (int)N, CUBLAS_COMPUTE_32F,
-                                          CUBLAS_GEMM_DEFAULT);
-    if (s != CUBLAS_STATUS_SUCCESS) {
-        set_error("cublasGemmEx failed (status %d)", (int)s);
-        return SQ_ERR_CUDA;
-    }
-    return SQ_OK;
+    return float_gemm_xwt(x, w, dt, T, N, K, yref, st);
 }
 
 }  // namespace

@@ -15,13 +15,14 @@ import re
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libsq.so")
+# SQ_LIBRARY=debug loads the -DSQ_DEBUG build (index checks in the kernels)
+LIB_PATH = os.path.join(_PKG, "libsq_debug.so" if os.environ.get("SQ_LIBRARY") == "debug" else "libsq.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "sq.h")
 
-SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
+SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT, SQ_ERR_BOUNDS = 0, 1, 2, 3, 4, 5
 SQ_F32, SQ_BF16, SQ_I32 = 0, 1, 2
 STATUS_NAMES = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED", 3: "SQ_ERR_CUDA",
-                4: "SQ_ERR_TIMEOUT"}
+                4: "SQ_ERR_TIMEOUT", 5: "SQ_ERR_BOUNDS"}
 
 
 class SqError(RuntimeError):
@@ -31,8 +32,9 @@ class SqError(RuntimeError):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libsq.so is not built ({LIB_PATH}); run "
-                      "`python -m w8a8_post_quantization_calibrate_b200.build`")
+    raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
+                      "`python -m w8a8_post_quantization_calibrate_b200.build`"
+                      + (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
 
 _lib = ctypes.CDLL(LIB_PATH)
 _vp, _i64, _f32, _sz, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_int
@@ -64,12 +66,15 @@ _SIGS = {
     "sq_w8a8_gemm": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp], _int),
     "sq_w8a8_gemm_noalloc": ([_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _int, _vp], _int),
     "sq_linear_workspace_size": ([_i64, _i64, _i64, _int, _int], _sz),
+    "sq_linear_workspace_offsets": ([_i64, _i64, _i64, _int, _int, _vp], _int),
     "sq_linear": ([_vp, _vp, _int, _i64, _i64, _i64, _f32, _f32, _vp, _int, _vp, _sz, _vp], _int),
     "sq_get_status": ([_vp], _int),
     "sq_last_status_site": ([], ctypes.c_uint),
     "sq_last_error_string": ([], ctypes.c_char_p),
     "sq_set_wait_timeout_ms": ([_i64], _int),
     "sq_selftest_wait_timeout": ([_i64, _vp], _int),
+    "sq_selftest_dirty_noalloc_scratch": ([_vp], _int),
+    "sq_probe_tensor_int8": ([_i64, _vp, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -364,13 +369,22 @@ def sq_w8a8_gemm_noalloc(xq: torch.Tensor, x_scale: torch.Tensor | None, wq: tor
     callers); the C call itself allocates nothing."""
     M, K = xq.shape
     N = wq.shape[0]
-    if y is None:
-        y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
-    _check(_lib.sq_w8a8_gemm_noalloc(_dev(xq, "xq"), x_scale.data_ptr() if x_scale is not None else None,
-                                     _dev(wq, "wq"), w_scale.data_ptr() if w_scale is not None else None,
-                                     M, N, K, _dev(y, "y"), _dt(y), _stream(stream)),
-           "sq_w8a8_gemm_noalloc")
+    for name, t in (("wq", wq), ("x_scale", x_scale), ("w_scale", w_scale), ("y", y)):
+        if t is not None and t.device != xq.device:
+            raise ValueError(f"{name} is on {t.device}, xq on {xq.device}")
+    # the C call takes the scratch of the current device: make it xq's
+    with torch.cuda.device(xq.device):
+        if y is None:
+            y = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+        _check(_lib.sq_w8a8_gemm_noalloc(_dev(xq, "xq"), x_scale.data_ptr() if x_scale is not None else None,
+                                         _dev(wq, "wq"), w_scale.data_ptr() if w_scale is not None else None,
+                                         M, N, K, _dev(y, "y"), _dt(y), _stream(stream)),
+               "sq_w8a8_gemm_noalloc")
     return y
+
+
+def sq_selftest_dirty_noalloc_scratch(stream=None) -> None:
+    _check(_lib.sq_selftest_dirty_noalloc_scratch(_stream(stream)), "sq_selftest_dirty_noalloc_scratch")
 
 
 def sq_outlier_split(xmax: torch.Tensor, threshold: float, keep: torch.Tensor | None = None,
@@ -459,6 +473,37 @@ def sq_linear_workspace_size(M: int, N: int, K: int, in_dtype=torch.bfloat16, ou
                                              _dt(torch.empty(0, dtype=out_dtype))))
 
 
+LINEAR_WORKSPACE_PARTS = ("xmax", "wmax", "s", "xq", "x_scale", "wq", "w_scale")
+
+
+def sq_linear_workspace_offsets(M: int, N: int, K: int, in_dtype=torch.bfloat16,
+                                out_dtype=torch.bfloat16) -> dict:
+    """Byte offsets of sq_linear's intermediates inside its workspace."""
+    off = (ctypes.c_size_t * len(LINEAR_WORKSPACE_PARTS))()
+    _check(_lib.sq_linear_workspace_offsets(M, N, K, _dt(torch.empty(0, dtype=in_dtype)),
+                                            _dt(torch.empty(0, dtype=out_dtype)), ctypes.cast(off, _vp)),
+           "sq_linear_workspace_offsets")
+    return dict(zip(LINEAR_WORKSPACE_PARTS, (int(v) for v in off)))
+
+
+def sq_linear_workspace_views(workspace: torch.Tensor, M: int, N: int, K: int, in_dtype=torch.bfloat16,
+                              out_dtype=torch.bfloat16) -> dict:
+    """Tensor views of sq_linear's intermediates (maxima, factors, codes and
+    scales) inside a workspace it has used."""
+    off = sq_linear_workspace_offsets(M, N, K, in_dtype, out_dtype)
+    shapes = {"xmax": ((K,), torch.float32), "wmax": ((K,), torch.float32), "s": ((K,), torch.float32),
+              "xq": ((M, K), torch.int8), "x_scale": ((M,), torch.float32),
+              "wq": ((N, K), torch.int8), "w_scale": ((N,), torch.float32)}
+    views = {}
+    for name, (shape, dt) in shapes.items():
+        n = 1
+        for d in shape:
+            n *= d
+        nbytes = n * torch.empty(0, dtype=dt).element_size()
+        views[name] = workspace[off[name]:off[name] + nbytes].view(dt).view(shape)
+    return views
+
+
 def sq_linear(x: torch.Tensor, w: torch.Tensor, alpha: float, eps: float = 1e-8,
               out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -501,6 +546,15 @@ def sq_set_wait_timeout_ms(ms: int) -> None:
 
 def sq_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     _check(_lib.sq_selftest_wait_timeout(int(limit_us), _stream(stream)), "sq_selftest_wait_timeout")
+
+
+def sq_probe_tensor_int8(iters: int, stream=None) -> float:
+    """Launch the int8 tensor-core rate probe; returns the int8 operations the
+    launch performs (time it with CUDA events on the stream)."""
+    ops = ctypes.c_double(0.0)
+    _check(_lib.sq_probe_tensor_int8(int(iters), ctypes.cast(ctypes.pointer(ops), _vp), _stream(stream)),
+           "sq_probe_tensor_int8")
+    return float(ops.value)
 
 
 def raw_status(fn_name: str, *args) -> int:
