@@ -441,20 +441,46 @@ def build_step(variant, sq, wl, x, w, xcal, dev, stream):
 
 def int8_probe(sq, dev, stream, clk, launches=PROBE_LAUNCHES, iters=PROBE_ITERS):
     """The int8 tensor-core rate (sq_probe_tensor_int8), median over launches
-    with CUDA events on the launching stream -> dict."""
+    with CUDA events on the launching stream, and the SM clock each launch ran
+    at (cycles over nanoseconds, measured by the kernel on one SM) -> dict."""
     clk.mark("probe")
-    times, ops = [], 0.0
+    times, mhz, ops = [], [], 0.0
+    clocks = torch.zeros(2, dtype=torch.int64, device=dev)
     for i in range(launches + 3):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        ops = sq.sq_probe_tensor_int8(iters, stream=stream)
+        ops = sq.sq_probe_tensor_int8(iters, clocks=clocks, stream=stream)
         b.record(stream)
         b.synchronize()
         if i >= 3:
             times.append(a.elapsed_time(b))
+            cyc, ns = (int(v) for v in clocks.tolist())
+            mhz.append(1e3 * cyc / ns if ns > 0 else float("nan"))
     ms = median(times)
-    return {"tops": ops / (ms * 1e-3) / 1e12, "ms": ms, "ops_per_launch": ops, "launches": launches,
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tops = ops / (ms * 1e-3) / 1e12
+    f = median(mhz)
+    return {"tops": tops, "ms": ms, "ops_per_launch": ops, "launches": launches, "sm_mhz_measured": round(f, 1),
+            "ops_per_sm_cycle": round(tops * 1e12 / (sms * f * 1e6), 1),
             "instruction": "tcgen05.mma.cta_group::2.kind::i8 256x256x32 from shared memory, every SM pair"}
+
+
+def gemm_sustained(stages, stream, clk, launches=30):
+    """The step's GEMM alone, back to back for `launches` launches, with the
+    SM clock sampled meanwhile (the clock the GEMM runs at under its own power
+    draw) -> (median ms per launch, clock summary)."""
+    fn = [f for n, f, _, _ in stages if n == "a5_w8a8_gemm"][0]
+    fn()
+    torch.cuda.synchronize()
+    clk.mark("gemm")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(launches + 1)]
+    ev[0].record(stream)
+    for i in range(launches):
+        fn()
+        ev[i + 1].record(stream)
+    ev[-1].synchronize()
+    clk.mark("between")
+    return median([ev[i].elapsed_time(ev[i + 1]) for i in range(launches)]), clk.summary({"gemm"})
 
 
 def int_mm_probe(dev, stream, n=8192, reps=10):
@@ -551,8 +577,10 @@ def run_ours(args, world, rank, local):
             clk.mark("sweep")
             sweep = alpha_sweep(sq, bufs, stages, x, w, stream, flush_l2, args.sweep_steps)
             clk.mark("between")
-        probe = int8_probe(sq, dev, stream, clk) if M > 16 else None
+        probe = int8_probe(sq, dev, stream, clk) if M > 16 and args.variant != "alpha_search" else None
         clk.mark("between")
+        sustained = (gemm_sustained(stages, stream, clk) if M > 16 and args.variant != "alpha_search"
+                     else (None, None))
     barrier(world)
     status = sq.sq_get_status(stream)
     if status != sq.SQ_OK:
@@ -608,9 +636,9 @@ def run_ours(args, world, rank, local):
                     "frac": round(achieved / int8_peak, 4),
                     "traffic": load_traffic(args.workload) if (M > 128 and default_gemm) else None,
                     "peak_source": ("measured int8: sq_probe_tensor_int8 in this run (median of "
-                                    f"{probe['launches']} launches of {probe['ms']:.3f} ms), SM clock median "
-                                    f"{clocks_p.get('sm_mhz')} MHz during the probe, "
-                                    f"{clocks_k.get('sm_mhz')} MHz during the kernel pass" if probe else
+                                    f"{probe['launches']} launches of {probe['ms']:.3f} ms at "
+                                    f"{probe['sm_mhz_measured']} MHz measured in the kernel); SM clock median "
+                                    f"{clocks_k.get('sm_mhz')} MHz (NVML) during the kernel pass" if probe else
                                     f"{peak_src}: bf16 x {INT8_OVER_BF16}"),
                     "peak_bf16x2": round(int8_from_bf16, 1),
                     "frac_of_bf16x2": round(achieved / int8_from_bf16, 4),
@@ -618,6 +646,17 @@ def run_ours(args, world, rank, local):
                                      f"int8/bf16 ratio",
                     "peak_spec": SPEC_INT8_TOPS, "frac_of_spec": round(achieved / SPEC_INT8_TOPS, 4),
                     "algorithmic_ops_per_launch": ops}
+        if probe and sustained[0] and sustained[1].get("sm_mhz"):
+            # per clock: the GEMM's ops per SM cycle (its back-to-back time at the
+            # clock sampled while it alone ran) over the probe's (its own clock)
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            g_tops = ops / (sustained[0] * 1e-3) / 1e12
+            g_opc = g_tops * 1e12 / (sms * sustained[1]["sm_mhz"] * 1e6)
+            roofline["per_clock"] = {"gemm_back_to_back_ms": round(sustained[0], 5), "gemm_tops": round(g_tops, 1),
+                                     "gemm_sm_mhz": sustained[1]["sm_mhz"], "gemm_ops_per_sm_cycle": round(g_opc, 1),
+                                     "probe_ops_per_sm_cycle": probe["ops_per_sm_cycle"],
+                                     "frac": round(g_opc / probe["ops_per_sm_cycle"], 4),
+                                     "gemm_clock_reasons": sustained[1].get("reasons")}
     else:
         gemm_ms = per_kernel["a5_w8a8_gemm"]
         gbs = kb["a5_w8a8_gemm"] / (gemm_ms * 1e-3) / 1e9
@@ -699,7 +738,7 @@ def run_ours(args, world, rank, local):
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu_baseline, "e2e": e2e,
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary({"steps", "kernels", "sweep"}),
-        "clocks_by_phase": {p: clk.summary({p}) for p in ("steps", "kernels", "sweep", "probe")},
+        "clocks_by_phase": {p: clk.summary({p}) for p in ("steps", "kernels", "sweep", "probe", "gemm")},
     }
     if probe:
         out["int8_probe"] = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in probe.items()}

@@ -433,8 +433,12 @@ sq_status sq_linear(const void* x, const void* w, sq_dtype in_dt, int64_t M, int
  * shared memory, with no global-memory traffic. *ops (host, may be NULL)
  * receives the int8 operations the launch performs (2 per multiply-add); the
  * caller times the launch (for example with CUDA events on `stream`).
+ * clocks (device, 2 entries, may be NULL) receives, from one SM, the SM clock
+ * cycles and the nanoseconds (%globaltimer) spanning its MMAs, so that the
+ * rate can be stated per cycle at the clock the launch ran at.
  * iters in [1, 10^7], else SQ_ERR_INVALID_ARG. Computes nothing else. */
-sq_status sq_probe_tensor_int8(int64_t iters, double* ops, sq_stream_t stream);
+sq_status sq_probe_tensor_int8(int64_t iters, double* ops, unsigned long long* clocks,
+                               sq_stream_t stream);
 
 /* ---------------------------------------------------------------- status
  * Synchronize `stream`, then return and clear the first error any kernel of

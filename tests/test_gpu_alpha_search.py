@@ -4,8 +4,12 @@
 Bar: every quantized output Yq(alpha) is the bit-exact fp32 path (checked by
 the other tests), so the errors differ only through the reference product Y
 (fp32-accumulated on the GPU, fp64 in the oracle) and the order of the fp64
-sums: relative difference below 1e-3, written in the test, and the same best
-alpha.
+sums. With fp32 operands the GPU's Y is a chain of fp32 fused multiply-adds in
+k order; with bf16 operands every product is exact and the tensor cores add
+them in fp32 in their own order. A relative error d in Y moves an error e by at
+most about d (1 + e): the differences seen on these cases are <= 7e-7 of e
+(fp32) and <= 2e-5 (bf16, K = 16384), and the tests allow 1e-5 and 1e-4, with
+the same best alpha.
 """
 import numpy as np
 import pytest
@@ -23,6 +27,7 @@ if not torch.cuda.is_available():
 from w8a8_post_quantization_calibrate_b200 import sq  # noqa: E402
 
 DEV = torch.device("cuda", 0)
+RTOL = {torch.float32: 1e-5, torch.bfloat16: 1e-4}
 
 
 def test_alpha_search_reproduces_the_alpha_table():
@@ -37,12 +42,12 @@ def test_alpha_search_reproduces_the_alpha_table():
     assert [round(100 * e, 1) for e in errs] == [row["error_percent"] for row in g["alpha_table"]], errs
     assert best == 0.5
     o_errs, o_best = oracle.alpha_search(X.astype(np.float32), W.astype(np.float32), alphas)
-    np.testing.assert_allclose(errs, o_errs, rtol=1e-3)
+    np.testing.assert_allclose(errs, o_errs, rtol=RTOL[torch.float32])
     assert o_best == best
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("T,N,K", [(8, 300, 272), (100, 520, 1040), (512, 1024, 4096)])
+@pytest.mark.parametrize("T,N,K", [(8, 300, 272), (100, 520, 1040), (512, 1024, 4096), (256, 512, 16384)])
 def test_alpha_search_matches_oracle(dtype, T, N, K):
     g = torch.Generator().manual_seed(T + N)
     x = torch.randn(T, K, generator=g)
@@ -52,8 +57,8 @@ def test_alpha_search_matches_oracle(dtype, T, N, K):
     alphas = [0.0, 0.25, 0.4, 0.5, 0.6, 0.75, 0.85, 1.0]
     errs, best = sq.sq_alpha_search(x.to(DEV), w.to(DEV), alphas)
     o_errs, o_best = oracle.alpha_search(synth.host_array(x), synth.host_array(w), alphas)
-    np.testing.assert_allclose(errs, o_errs, rtol=1e-3)
-    assert best == o_best or abs(o_errs[alphas.index(best)] - min(o_errs)) <= 1e-3 * min(o_errs)
+    np.testing.assert_allclose(errs, o_errs, rtol=RTOL[dtype])
+    assert best == o_best or abs(o_errs[alphas.index(best)] - min(o_errs)) <= RTOL[dtype] * min(o_errs)
     assert sq.sq_get_status() == sq.SQ_OK
 
 

@@ -187,8 +187,8 @@ def test_keep_mask_fold_is_the_bulk_quantizer():
     assert_bitexact_f32(host(sc), osc, "bulk scales")
 
 
-# (300, 200, 28672) and (200, 100, 16400): 16-warp rows (multipliers in
-# registers), with CTAs whose rows run from the weights into the activations.
+# (300, 200, 28672) and (200, 100, 16400): 16-warp rows, enough rows that
+# CTAs run from the weights into the activations where the pair is one launch.
 PAIR_SHAPES = [(300, 37, 4096), (1000, 7, 4112), (70, 90, 5120), (64, 200, 6160), (5, 900, 4096), (50, 3, 16384),
                (9, 5, 28672), (300, 200, 28672), (200, 100, 16400), (40, 33, 2048)]
 
@@ -197,8 +197,9 @@ PAIR_SHAPES = [(300, 37, 4096), (1000, 7, 4112), (70, 90, 5120), (64, 200, 6160)
 @pytest.mark.parametrize("N,T,K", PAIR_SHAPES)
 def test_pair_launch_equals_the_two_calls(dtype, N, T, K):
     """a3 and a4 in one launch (weights' rows, then activations' rows): the
-    same codes and scales as the two calls and as the oracle. K = 2048 or
-    fp32 rows (outside the streamed kernel) take the two calls."""
+    same codes and scales as the two calls and as the oracle. K = 28672 (two
+    multiplier tables do not fit beside the ring) and K = 2048 or fp32 rows
+    (outside the streamed kernel) take the two calls."""
     g = torch.Generator().manual_seed(N + T + K)
     w = (torch.randn(N, K, generator=g) * 0.05).to(dtype)
     x = outlier_x(T, K, seed=N * 7 + K).to(dtype)

@@ -131,6 +131,59 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, l
     }
 }
 
+// ---------------------------------------------------------------- thread-block clusters
+// Rank of this CTA in its cluster, the cluster's size, a barrier of all the
+// cluster's threads, and the cluster-scope pieces of an exchange between CTAs:
+// the shared::cluster address of an offset in another CTA, an integer atomic
+// add there, a remote arrive that releases this thread's earlier writes, and a
+// bounded wait that acquires them.
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t local_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void red_add_cluster(uint32_t cluster_addr, int32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.add.s32 [%0], %1;" :: "r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void arrive_remote_release(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_acq_cluster(uint32_t bar, uint32_t parity, long long limit,
+                                                      volatile int* abort, unsigned int site) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit) {
+            *abort = 1;
+            record_status(SQ_ERR_TIMEOUT, site);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // The library's kernels are launched with programmatic stream serialization:
 // a kernel may be scheduled while the previous kernel in the stream is still

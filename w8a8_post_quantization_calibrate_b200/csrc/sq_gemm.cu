@@ -444,14 +444,6 @@ constexpr size_t pair_smem_bytes() {
     return 1024 + P_STAGES * (P_A_STAGE + P_B_STAGE) + 256;
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cta0, int32_t x, int32_t y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -946,44 +938,6 @@ struct DecodeSplit {
     }
 };
 
-__device__ __forceinline__ uint32_t mapa_rank(uint32_t local_addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void red_add_cluster(uint32_t cluster_addr, int32_t v) {
-    asm volatile("red.relaxed.cluster.shared::cluster.add.s32 [%0], %1;" :: "r"(cluster_addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void arrive_remote_release(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_acq_cluster(uint32_t bar, uint32_t parity, long long limit,
-                                                      volatile int* abort, unsigned int site) {
-    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_try_wait_acq_cluster(bar, parity)) return true;
-        if (*abort) return false;
-        if (clock64() - t0 > limit) {
-            *abort = 1;
-            record_status(SQ_ERR_TIMEOUT, site);
-            return false;
-        }
-    }
-}
-__device__ __forceinline__ uint32_t cluster_nctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-    return r;
-}
 
 constexpr size_t DC_RECV_BYTES = (size_t)S_BN * S_BM * sizeof(int32_t);   // 8 KB: [token][row] int32
 constexpr size_t decode_cluster_smem_bytes() {

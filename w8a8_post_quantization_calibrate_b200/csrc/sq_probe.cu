@@ -24,8 +24,14 @@ constexpr uint32_t PROBE_TILE = 128 * BK;  // 16 KB: 128 rows x 128 bytes
 constexpr size_t PROBE_SMEM = 140 * 1024;
 constexpr int64_t PROBE_MAX_ITERS = 10000000;
 
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 __global__ void __launch_bounds__(PROBE_THREADS, 1)
-probe_mma_i8_pair_kernel(int64_t iters, long long wait_limit) {
+probe_mma_i8_pair_kernel(int64_t iters, long long wait_limit, unsigned long long* __restrict__ clocks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -57,6 +63,8 @@ probe_mma_i8_pair_kernel(int64_t iters, long long wait_limit) {
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
+    const long long c0 = clock64();
+    const unsigned long long t0 = global_ns();
     if (warp == 0 && lane == 0 && rank == 0) {
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
         for (int64_t it = 0; it < iters; ++it) {
@@ -69,6 +77,11 @@ probe_mma_i8_pair_kernel(int64_t iters, long long wait_limit) {
         mma_commit_pair(smem_u32(done));   // arrives on both CTAs' barrier once every MMA is done
     }
     if (warp == 0 && lane == 0) mbar_wait(smem_u32(done), 0, wait_limit, &abort_flag, SITE_PROBE);
+    if (clocks != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+        // this SM's clock over the MMAs: cycles and nanoseconds
+        clocks[0] = (unsigned long long)(clock64() - c0);
+        clocks[1] = global_ns() - t0;
+    }
     __syncwarp();
     tc_fence_before();
     cluster_sync_all();
@@ -78,7 +91,7 @@ probe_mma_i8_pair_kernel(int64_t iters, long long wait_limit) {
     }
 }
 
-sq_status probe_tensor_int8(int64_t iters, double* ops, cudaStream_t st) {
+sq_status probe_tensor_int8(int64_t iters, double* ops, unsigned long long* clocks, cudaStream_t st) {
     if (iters < 1 || iters > PROBE_MAX_ITERS) {
         set_error("iters=%lld must be in [1, %lld]", (long long)iters, (long long)PROBE_MAX_ITERS);
         return SQ_ERR_INVALID_ARG;
@@ -91,7 +104,7 @@ sq_status probe_tensor_int8(int64_t iters, double* ops, cudaStream_t st) {
     // the MMAs of one launch, plus a margin, within the bounded wait
     const long long limit = wait_limit_cycles() + iters * 4 * 2000LL;
     r = launch_pdl("probe_mma_i8_pair_kernel", probe_mma_i8_pair_kernel, dim3(2 * pairs), dim3(PROBE_THREADS),
-                   PROBE_SMEM, st, 2, iters, limit);
+                   PROBE_SMEM, st, 2, iters, limit, clocks);
     if (r != SQ_OK) return r;
     if (ops) *ops = 2.0 * 256.0 * 256.0 * (double)UMMA_K * (BK / UMMA_K) * (double)iters * (double)pairs;
     return SQ_OK;
@@ -99,6 +112,7 @@ sq_status probe_tensor_int8(int64_t iters, double* ops, cudaStream_t st) {
 
 }  // namespace sq
 
-extern "C" sq_status sq_probe_tensor_int8(int64_t iters, double* ops, sq_stream_t stream) {
-    return sq::probe_tensor_int8(iters, ops, (cudaStream_t)stream);
+extern "C" sq_status sq_probe_tensor_int8(int64_t iters, double* ops, unsigned long long* clocks,
+                                          sq_stream_t stream) {
+    return sq::probe_tensor_int8(iters, ops, clocks, (cudaStream_t)stream);
 }

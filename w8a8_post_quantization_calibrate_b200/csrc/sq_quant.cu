@@ -768,8 +768,7 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
 // maximum is always among them, since m' <= a(1 + 3 * 2^-24) and the element
 // attaining a has |v'| >= a(1 - 3 * 2^-24). (Resolving candidates against
 // each lane's own maximum instead saves the second group reduction but puts an
-// IEEE division in every lane: measured slower at K = 4096, 23.4 against
-// 20.5 us.)
+// IEEE division in every lane: measured slower, 20.5 -> 22.5 us at K = 4096.)
 //
 // Codes (pass 2): with r = RN(1/scale), t = RN(v * r + 1.5 * 2^23) holds
 // k = round-half-even(v * r) in its low mantissa bits, and d = RN(v * r - k)
@@ -833,13 +832,7 @@ struct RingPair {
     float* scale2 = nullptr;
 };
 
-// MREG (rows of 16 warps, K > 16384): each lane keeps the multipliers of its
-// CPL chunks in registers (a lane owns the same chunks in every row) instead of
-// a CTA-wide table in shared memory, and pass 2 recomputes the values from the
-// row still in its slot; the 114 KB a table takes at K = 28672 go to ring
-// slots instead (three rows in flight per CTA, and a pair launch fits). The
-// values, and so every result, are the same as with the table.
-template <int MODE, int R, int CPL, bool FULL, bool PAIR, int FMT, bool MREG = false>
+template <int MODE, int R, int CPL, bool FULL, bool PAIR, int FMT>
 __global__ void __launch_bounds__(kRingThreads, 1)
 row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t K, const float* __restrict__ s,
                       int8_t* __restrict__ q, float* __restrict__ scale_out, float eps, float* __restrict__ r_out,
@@ -858,7 +851,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
     float* mul_hi = mul_lo + NCP * 4;                            // [NCP][4]: elements 4..7
     float* mul2_lo = mul_hi + NCP * 4;                           // PAIR: RN(1/s_j) for the second tensor
     float* mul2_hi = mul2_lo + NCP * 4;
-    uint8_t* slots = ring_smem + (MREG ? 0 : NCP * (PAIR ? 64 : 32));   // [G][ns][SLOT]
+    uint8_t* slots = ring_smem + NCP * (PAIR ? 64 : 32);         // [G][ns][SLOT]
     uint64_t* bars = reinterpret_cast<uint64_t*>(slots + (size_t)G * ns * SLOT);   // [G][ns]
     float* red = reinterpret_cast<float*>(bars + G * ns);        // [G][2][R]
     double* red64 = reinterpret_cast<double*>(red + G * 2 * R);  // [G][2][R]
@@ -887,39 +880,21 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
     };
     const int64_t stride = (int64_t)gridDim.x * G;
     const int64_t row0 = (int64_t)blockIdx.x * G + grp;
+    int issued = 0;   // copies this group has issued (rows row0 + j * stride, j < issued)
     if (gl == 0) {
         for (int j = 0; j < ns; ++j) {
             const int64_t row = row0 + (int64_t)j * stride;
             if (row < total) {
                 mbar_arrive_expect_tx(bar0 + 8u * j, row_bytes);
                 bulk_copy_g2s(smem_u32(my_slots + (size_t)j * SLOT), row_src(row), row_bytes, bar0 + 8u * j);
+                ++issued;
             }
         }
     }
     // multipliers, zero past the row's end; the slots' padding (never
     // written by a copy) is zeroed once, so every lane handles CPL chunks
     // without bounds checks and the padding adds nothing to any maximum
-    float mr[MREG ? CPL : 1][8];     // MREG: this lane's multipliers
-    bool mr_second = false;          // MREG pair launch: mr holds the second tensor's RN(1/s_j)
-    auto load_mr = [&](bool recip) {
-#pragma unroll
-        for (int i = 0; i < (MREG ? CPL : 1); ++i) {
-            const int c = gl + i * 32 * R;
-            float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f), b = a;
-            if (c < nch) {
-                a = __ldg(reinterpret_cast<const float4*>(s + c * 8));
-                b = __ldg(reinterpret_cast<const float4*>(s + c * 8 + 4));
-                if (recip) {
-                    a = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
-                    b = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
-                }
-            }
-            mr[i][0] = a.x; mr[i][1] = a.y; mr[i][2] = a.z; mr[i][3] = a.w;
-            mr[i][4] = b.x; mr[i][5] = b.y; mr[i][6] = b.z; mr[i][7] = b.w;
-        }
-    };
-    if (MREG) load_mr(MODE == kSmooth);
-    for (int c = threadIdx.x; c < (MREG ? 0 : NCP); c += kRingThreads) {
+    for (int c = threadIdx.x; c < NCP; c += kRingThreads) {
         float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f), b = a;
         if (c < nch) {
             a = __ldg(reinterpret_cast<const float4*>(s + c * 8));
@@ -962,10 +937,6 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         float* const so = second ? pr.scale2 : scale_out;
         const float* const mlo = second ? mul2_lo : mul_lo;
         const float* const mhi = second ? mul2_hi : mul_hi;
-        if (MREG && PAIR && second && !mr_second) {
-            load_mr(true);   // from here on this group quantizes the second tensor
-            mr_second = true;
-        }
         const bool ok = mbar_wait_sleep(bar0 + 8u * sl, parity, wait_limit, &abort_sh, SITE_QUANT_WAIT);
         __syncwarp();   // the barrier below is warp-aligned
         if (!group_all<R>(ok, grp)) {
@@ -978,6 +949,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             if (nr < total) {
                 mbar_arrive_expect_tx(bar0 + 8u * ps, row_bytes);
                 bulk_copy_g2s(smem_u32(my_slots + (size_t)ps * SLOT), row_src(nr), row_bytes, bar0 + 8u * ps);
+                ++issued;
             }
         }
         const uint8_t* src = my_slots + (size_t)sl * SLOT;
@@ -1009,42 +981,24 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         const uint64_t rn2 = f2_pack(rn, rn);
 
         // ---- pass 1: the values, kept in registers, and their maximum
-        // (MREG: the values are recomputed in pass 2 instead of kept)
-        uint64_t v2[MREG ? 1 : CPL][4];
+        uint64_t v2[CPL][4];
         float cm[CPL];
         float m = 0.0f;
-        // multipliers of chunk i as fp32 pairs: from registers (MREG) or the table
-        auto mpairs = [&](int i, int c, uint64_t (&mp)[4]) {
-            if (MREG) {
-                const int ii = MREG ? i : 0;
-                mp[0] = f2_pack(mr[ii][0], mr[ii][1]);
-                mp[1] = f2_pack(mr[ii][2], mr[ii][3]);
-                mp[2] = f2_pack(mr[ii][4], mr[ii][5]);
-                mp[3] = f2_pack(mr[ii][6], mr[ii][7]);
-            } else {
-                const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
-                const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
-                mp[0] = f2_pack(a.x, a.y);
-                mp[1] = f2_pack(a.z, a.w);
-                mp[2] = f2_pack(b.x, b.y);
-                mp[3] = f2_pack(b.z, b.w);
-            }
-        };
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
             const int c = gl + i * 32 * R;
             const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-            uint64_t mp[4];
-            mpairs(i, c, mp);
+            const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
+            const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
+            const uint64_t mp[4] = {f2_pack(a.x, a.y), f2_pack(a.z, a.w), f2_pack(b.x, b.y), f2_pack(b.z, b.w)};
             float cmax = 0.0f;
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
                 uint64_t x2 = bf16_pair(w, p);
                 if (MODE == kNorm) x2 = f2_mul(x2, rn2);
-                const uint64_t vv = f2_mul(x2, mp[p]);
-                if (!MREG) v2[MREG ? 0 : i][p] = vv;
+                v2[i][p] = f2_mul(x2, mp[p]);
                 float lo, hi;
-                f2_unpack(vv, lo, hi);
+                f2_unpack(v2[i][p], lo, hi);
                 cmax = fmax3(cmax, fabsf(lo), fabsf(hi));
             }
             cm[i] = cmax;
@@ -1097,7 +1051,6 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             continue;
         }
 
-
         if (smooth) {
             // exact values of the candidates (normally the maximum alone)
             const float thr = __fmul_rn(amax, kRingCandidate);
@@ -1105,35 +1058,18 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
 #pragma unroll
             for (int i = 0; i < CPL; ++i) cand |= (cm[i] >= thr ? 1u : 0u) << i;
             float ex = 0.0f;
-            if (MREG) {
-                // statically unrolled: the register multipliers are indexed by i
+            while (cand) {
+                const int i = __ffs(cand) - 1;
+                cand &= cand - 1;
+                const int c = gl + i * 32 * R;
+                const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
+                const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
+                const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
+                const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-                for (int i = 0; i < CPL; ++i) {
-                    if (!(cand & (1u << i))) continue;
-                    const int c = gl + i * 32 * R;
-                    const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float x = bf16_elem(w, e);
-                        if (fabsf(__fmul_rn(x, mr[MREG ? i : 0][e])) >= thr)
-                            ex = fmaxf(ex, exact_abs<kSmooth>(x, __ldg(s + c * 8 + e), rn));
-                    }
-                }
-            } else {
-                while (cand) {
-                    const int i = __ffs(cand) - 1;
-                    cand &= cand - 1;
-                    const int c = gl + i * 32 * R;
-                    const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-                    const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
-                    const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
-                    const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float x = bf16_elem(w, e);
-                        if (fabsf(__fmul_rn(x, mv[e])) >= thr)
-                            ex = fmaxf(ex, exact_abs<kSmooth>(x, __ldg(s + c * 8 + e), rn));
-                    }
+                for (int e = 0; e < 8; ++e) {
+                    const float x = bf16_elem(w, e);
+                    if (fabsf(__fmul_rn(x, mv[e])) >= thr) ex = fmaxf(ex, exact_abs<kSmooth>(x, __ldg(s + c * 8 + e), rn));
                 }
             }
             amax = group_max<R>(ex, red, grp, wig, lane, bank);
@@ -1151,26 +1087,10 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             for (int i = 0; i < CPL; ++i) {
                 uint32_t t[8];
                 float dm = 0.0f;
-                uint64_t vi[4];
-                if (MREG) {
-                    const int c = gl + i * 32 * R;
-                    const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-                    uint64_t mp[4];
-                    mpairs(i, c, mp);
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        uint64_t x2 = bf16_pair(w, p);
-                        if (MODE == kNorm) x2 = f2_mul(x2, rn2);
-                        vi[p] = f2_mul(x2, mp[p]);
-                    }
-                } else {
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) vi[p] = v2[MREG ? 0 : i][p];
-                }
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const uint64_t t2 = f2_fma(vi[p], r2, mag2);
-                    const uint64_t d2 = f2_fma(vi[p], r2, f2_sub(mag2, t2));
+                    const uint64_t t2 = f2_fma(v2[i][p], r2, mag2);
+                    const uint64_t d2 = f2_fma(v2[i][p], r2, f2_sub(mag2, t2));
                     float t0, t1, d0, d1;
                     f2_unpack(t2, t0, t1);
                     f2_unpack(d2, d0, d1);
@@ -1192,21 +1112,9 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             for (int i = 0; i < CPL; ++i) {
                 uint32_t c16[4];
                 uint32_t diff = 0;
-                uint64_t vi[4];
-                if (MREG) {
-                    const int c = gl + i * 32 * R;
-                    const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-                    uint64_t mp[4];
-                    mpairs(i, c, mp);
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) vi[p] = f2_mul(bf16_pair(w, p), mp[p]);
-                } else {
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) vi[p] = v2[MREG ? 0 : i][p];
-                }
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const uint64_t q2 = f2_mul(vi[p], r2);
+                    const uint64_t q2 = f2_mul(v2[i][p], r2);
                     float l0, l1, h0, h1;
                     f2_unpack(f2_mul(q2, lo2), l0, l1);
                     f2_unpack(f2_mul(q2, hi2), h0, h1);
@@ -1230,24 +1138,14 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         if (gl == 0 && dchk(row < trows, SITE_DBG_RING_SCALE)) so[row] = scale;
         // near ties: the same fast quotient recomputed per element; those
         // within the guard get the IEEE-division code (same thread, later store)
-        // (MREG: statically unrolled over the chunks, the multipliers from registers)
-#pragma unroll
-        for (int ii = 0; ii < (MREG ? CPL : 1); ++ii)
-        while (MREG ? ((ntm >> ii) & 1u) != 0 : ntm != 0) {
-            const int i = MREG ? ii : __ffs(ntm) - 1;
-            ntm &= MREG ? ~(1u << ii) : ntm - 1;
+        while (ntm) {
+            const int i = __ffs(ntm) - 1;
+            ntm &= ntm - 1;
             const int c = gl + i * 32 * R;
             const uint4 w = *reinterpret_cast<const uint4*>(src + c * 16);
-            float mv[8];
-            if (MREG) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) mv[e] = mr[MREG ? ii : 0][e];
-            } else {
-                const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
-                const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
-                mv[0] = a.x; mv[1] = a.y; mv[2] = a.z; mv[3] = a.w;
-                mv[4] = b.x; mv[5] = b.y; mv[6] = b.z; mv[7] = b.w;
-            }
+            const float4 a = *reinterpret_cast<const float4*>(mlo + c * 4);
+            const float4 b = *reinterpret_cast<const float4*>(mhi + c * 4);
+            const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float x = bf16_elem(w, e);
@@ -1272,10 +1170,8 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
     if (failed && gl == 0) {
         // copies issued for rows this group will not consume: let them land
         // before the CTA exits (bounded)
-        for (int j = it; j < it + ns - 1; ++j) {
-            const int64_t row = row0 + (int64_t)j * stride;
-            if (row < total) mbar_wait(bar0 + 8u * (j % ns), (uint32_t)(j / ns) & 1u, wait_limit, &never_sh, SITE_QUANT_DRAIN);
-        }
+        for (int j = it; j < issued; ++j)
+            mbar_wait(bar0 + 8u * (j % ns), (uint32_t)(j / ns) & 1u, wait_limit, &never_sh, SITE_QUANT_DRAIN);
     }
 }
 
@@ -1361,21 +1257,19 @@ sq_status launch_row_quant_fast_inst(const void* in, int64_t rows, int64_t K, co
 // The streamed kernel's shared memory: multipliers (two tables for a pair
 // launch) and ns row slots per group, both padded to 32 * R * CPL chunks, the
 // slots' mbarriers and the group reduction slots.
-size_t ring_smem_bytes(int R, int CPL, int ns, bool pair, bool mreg = false) {
+size_t ring_smem_bytes(int R, int CPL, int ns, bool pair) {
     const size_t G = (size_t)(kRingThreads / (32 * R));
     const size_t ncp = (size_t)32 * R * CPL;
-    return (mreg ? 0 : ncp * (pair ? 64 : 32)) + G * (size_t)ns * (ncp * 16 + 8) + G * 2 * (size_t)R * (4 + 8);
+    return ncp * (pair ? 64 : 32) + G * (size_t)ns * (ncp * 16 + 8) + G * 2 * (size_t)R * (4 + 8);
 }
 
 template <int MODE, int R, int CPL, bool FULL, bool PAIR, int FMT>
 sq_status launch_row_quant_ring_inst(const void* in, int64_t rows, int64_t K, const float* s, int8_t* q,
                                      float* scale, cudaStream_t st, float eps, float* r_out, int ns,
                                      const RingPair& pr) {
-    // rows of 16 warps keep their multipliers in registers
-    constexpr bool MREG = R == 16;
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
-    auto kern = row_quant_ring_kernel<MODE, R, CPL, FULL, PAIR, FMT, MREG>;
+    auto kern = row_quant_ring_kernel<MODE, R, CPL, FULL, PAIR, FMT>;
     if (!attr_done[di.device & 63]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row_quant_ring_kernel)");
@@ -1384,8 +1278,7 @@ sq_status launch_row_quant_ring_inst(const void* in, int64_t rows, int64_t K, co
     constexpr int G = kRingThreads / (32 * R);
     const int64_t need = (rows + (PAIR ? pr.rows2 : 0) + G - 1) / G;
     const int grid = (int)(need < di.sm_count ? need : di.sm_count);
-    return launch_pdl("row_quant_ring_kernel", kern, dim3(grid), dim3(kRingThreads),
-                      ring_smem_bytes(R, CPL, ns, PAIR, MREG),
+    return launch_pdl("row_quant_ring_kernel", kern, dim3(grid), dim3(kRingThreads), ring_smem_bytes(R, CPL, ns, PAIR),
                       st, 1, static_cast<const __nv_bfloat16*>(in), rows, K, s, q, scale, eps, r_out, ns,
                       wait_limit_cycles(), pr);
 }
@@ -1443,12 +1336,8 @@ bool launch_row_quant_ring(const void* in, int64_t rows, int64_t K, const float*
         R = 2;
         cpl = 10;
     }
-    // two ring slots per group (one row in flight while one is processed:
-    // measured faster than three or four); rows of 16 warps, whose
-    // multipliers live in registers, take three (one group per CTA)
-    const bool mreg = R == 16;
-    const int ns = mreg ? 3 : 2;
-    if (ring_smem_bytes(R, cpl, ns, PAIR, mreg) > kRingSmemMax) return false;
+    const int ns = 2;
+    if (ring_smem_bytes(R, cpl, ns, PAIR) > kRingSmemMax) return false;
     if (FMT != kInt8 && nchunks != (int64_t)32 * R * cpl) return false;
 #define SQ_RING_R(RR) launch_row_quant_ring_r<MODE, RR, PAIR, FMT>(cpl, in, rows, K, s, q, scale, st, eps, r_out, ns, pr)
     switch (R) {

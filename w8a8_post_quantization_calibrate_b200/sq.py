@@ -74,7 +74,7 @@ _SIGS = {
     "sq_set_wait_timeout_ms": ([_i64], _int),
     "sq_selftest_wait_timeout": ([_i64, _vp], _int),
     "sq_selftest_dirty_noalloc_scratch": ([_vp], _int),
-    "sq_probe_tensor_int8": ([_i64, _vp, _vp], _int),
+    "sq_probe_tensor_int8": ([_i64, _vp, _vp, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -548,11 +548,14 @@ def sq_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     _check(_lib.sq_selftest_wait_timeout(int(limit_us), _stream(stream)), "sq_selftest_wait_timeout")
 
 
-def sq_probe_tensor_int8(iters: int, stream=None) -> float:
+def sq_probe_tensor_int8(iters: int, clocks: torch.Tensor | None = None, stream=None) -> float:
     """Launch the int8 tensor-core rate probe; returns the int8 operations the
-    launch performs (time it with CUDA events on the stream)."""
+    launch performs (time it with CUDA events on the stream). `clocks`, a
+    CUDA int64 tensor of 2 entries if given, receives one SM's cycles and
+    nanoseconds over the MMAs."""
     ops = ctypes.c_double(0.0)
-    _check(_lib.sq_probe_tensor_int8(int(iters), ctypes.cast(ctypes.pointer(ops), _vp), _stream(stream)),
+    _check(_lib.sq_probe_tensor_int8(int(iters), ctypes.cast(ctypes.pointer(ops), _vp),
+                                     None if clocks is None else _dev(clocks, "clocks"), _stream(stream)),
            "sq_probe_tensor_int8")
     return float(ops.value)
 
