@@ -85,10 +85,10 @@ def load_traffic(workload: str):
         return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("source_sha256_16") != gemm_source_hash():
-        return None
     per = d.get("per_workload", {}).get(workload)
-    return None if per is None else per.get("dram_bytes_per_launch")
+    if per is None or per.get("source_sha256_16") != gemm_source_hash():
+        return None
+    return per.get("dram_bytes_per_launch")
 
 
 def dist_env():
