@@ -175,6 +175,41 @@ def test_tiny_denormal_zero_and_huge_rows():
         check_norm(x, gf, eps, f"extreme rows, norm eps={eps}")
 
 
+def _half_step_rows(K, seed):
+    """Raw bf16 rows whose maximum is 127 * 2^e, so the scale is the power of
+    two 2^e and every value (2k + 1) 2^(e - 1) is an exact half-step of the
+    grid: round half to even decides its code. Rows at e = -3 (values below
+    one), e = -60 and e = +40, and a row of N(0, 1) data (its own ties)."""
+    rng = np.random.default_rng(seed)
+    odd = (2 * rng.integers(0, 127, K) + 1).astype(np.float64) * rng.choice([-1.0, 1.0], K)
+    rows = []
+    for e in (-3, -60, 40):
+        r = odd * 2.0 ** (e - 1)
+        r[rng.integers(0, K)] = 127.0 * 2.0 ** e
+        rows.append(r)
+    rows.append(rng.standard_normal(K))
+    return torch.tensor(np.array(rows), dtype=torch.float64).to(BF16)
+
+
+@pytest.mark.parametrize("K", [512, 2048, 4096, 28672])
+def test_exact_half_steps_of_raw_bf16(K):
+    """Raw bf16 values on exact half-steps take the near-tie path of the fold
+    (multiplier 1 and a power of two), of the bulk quantizer (0/1 multiplier)
+    and of RMSNorm; K = 512 and 2048 run the register kernel, 4096 and 28672
+    the streamed one."""
+    x = _half_step_rows(K, K + 3)
+    hx = synth.host_array(x)
+    assert (x.float().abs() == 127.0 * 2.0 ** -3).any(), "the bf16 rows hold the maxima exactly"
+    check_fold(x, np.ones(K, np.float32), f"half steps, fold s=1, K={K}")
+    check_fold(x, np.full(K, 0.25, np.float32), f"half steps, fold s=1/4, K={K}")
+    keep = np.ones(K, np.float32)
+    keep[np.random.default_rng(K).choice(K, 5, replace=False)] = 0.0
+    q, sc = sq.sq_quant_bulk(dev(x), dev(torch.from_numpy(keep)))
+    oq, osc = oracle.quant_bulk(hx, keep)
+    assert_equal(host(q), oq, f"half steps, bulk codes K={K}")
+    assert_bitexact_f32(host(sc), osc, f"half steps, bulk scales K={K}")
+
+
 def test_keep_mask_fold_is_the_bulk_quantizer():
     """The decomposition's bulk quantizer (a 0/1 multiplier) on the streamed path."""
     K = 4096

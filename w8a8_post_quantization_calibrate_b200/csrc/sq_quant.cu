@@ -432,6 +432,30 @@ __device__ __noinline__ uint32_t exact_code(float x, float s_j, float scale, flo
     return (uint32_t)qi & 0xffu;
 }
 
+// The int8 code clamp(round_half_even(RN(v / scale)), -127, 127) of an exact
+// value v whose approximate quotient p (within 2^-15 of v / scale) lies within
+// 2^-13 of the half-integer h = floor(p) + 1/2, without a division. The true
+// quotient Q = v / scale is then within 2^-12 of h, so v - h * scale is a
+// multiple of 2^(e - 25) (e the exponent of scale; h a multiple of 1/2, v no
+// finer) below 2^(e - 11) in magnitude: exact in one fused multiply-add, and its
+// sign places Q against h. RN(Q) = h exactly when |Q - h| <= ulp(h) / 2, i.e.
+// when |v - h * scale| <= scale * ulp(h) / 2 (a product with a power of two,
+// exact); the equal case belongs to h because h, a multiple of 1/2 below 2^23,
+// has an even significand. A quotient that rounds to h takes h's even
+// neighbour (round half to even); any other lies strictly between h and the
+// integer on Q's side, which is its code. Requires scale >= 2^-100 (the
+// kernels send rows with smaller maxima to the exact path).
+__device__ __forceinline__ uint32_t near_tie_code(float v, float scale, float p) {
+    const int lo = __float2int_rd(p);
+    const float h = __fadd_rn((float)lo, 0.5f);
+    const float res = __fmaf_rn(-h, scale, v);
+    const uint32_t eh = (__float_as_uint(h) >> 23) & 0xffu;         // |h| >= 1/2: a normal number
+    const float bound = __fmul_rn(scale, __uint_as_float((eh - 24u) << 23));   // scale * ulp(h) / 2
+    int code = fabsf(res) <= bound ? lo + (lo & 1) : (res > 0.0f ? lo + 1 : lo);
+    code = max(-127, min(127, code));
+    return (uint32_t)code & 0xffu;
+}
+
 // The code of one element in either format (int8: as exact_code; E4M3: the
 // IEEE quotient converted with round-to-nearest-even and saturation).
 template <int MODE, int FMT>
@@ -460,18 +484,21 @@ __device__ __forceinline__ double group_sum(double v, double* red, int grp, int 
     return v;
 }
 
+// Maximum over the R <= 32 warps of a group. Every value is non-negative and
+// not NaN (maxima of |v| started from +0 with NaN-dropping max), so the bit
+// patterns order as the values do and integer warp reductions give the
+// maximum: one per warp, one slot per warp in shared memory, a named barrier,
+// one over the R slots.
 template <int R>
 __device__ __forceinline__ float group_max(float v, float* red, int grp, int wig, int lane, int bank) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (R == 1) return v;
-    float* slot = red + (grp * 2 + bank) * R;
-    if (lane == 0) slot[wig] = v;
+    static_assert(R >= 1 && R <= 32, "one slot per lane");
+    uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(v));
+    if (R == 1) return __uint_as_float(u);
+    uint32_t* slot = reinterpret_cast<uint32_t*>(red) + (grp * 2 + bank) * R;
+    if (lane == 0) slot[wig] = u;
     asm volatile("bar.sync %0, %1;" :: "r"(1 + grp), "r"(32 * R) : "memory");
-    v = slot[0];
-#pragma unroll
-    for (int w = 1; w < R; ++w) v = fmaxf(v, slot[w]);
-    return v;
+    u = lane < R ? slot[lane] : 0u;
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, u));
 }
 
 // The rarely taken paths of the row kernel. Kernels that keep one row in
@@ -519,10 +546,12 @@ __device__ __forceinline__ uint2 fix_near_ties_in(const RawChunk<T>& ch, uint2 c
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         const float xe = MODE == kNorm ? __fmul_rn(ch.get(e), rn) : ch.get(e);
-        const float qv = __fmul_rn(__fmul_rn(xe, mv[e]), r);
+        const float ve = __fmul_rn(xe, mv[e]);   // exact v for fold and norm
+        const float qv = __fmul_rn(ve, r);
         const float d = __fsub_rn(qv, __fsub_rn(__fadd_rn(qv, kMagic), kMagic));
         if (fabsf(d) >= 0.5f - kTieGuard) {
-            const uint32_t code = exact_code<MODE>(ch.get(e), __ldg(s8 + e), scale, rn);
+            const uint32_t code = MODE == kSmooth ? exact_code<MODE>(ch.get(e), __ldg(s8 + e), scale, rn)
+                                                  : near_tie_code(ve, scale, qv);
             const int sh = 8 * (e & 3);
             uint32_t& w = (e < 4) ? codes.x : codes.y;
             w = (w & ~(0xffu << sh)) | (code << sh);
@@ -1160,9 +1189,13 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                     redo = __nv_cvt_float_to_fp8(__fmul_rn(qf, 1.0f - 1.0f / 262144.0f), __NV_SATFINITE, __NV_E4M3) !=
                            __nv_cvt_float_to_fp8(__fmul_rn(qf, 1.0f + 1.0f / 262144.0f), __NV_SATFINITE, __NV_E4M3);
                 }
-                if (redo && dchk(c < nchunks, SITE_DBG_RING_REPAIR))
-                    rq[c * 8 + e] = (int8_t)(second ? exact_code_fmt<kSmooth, FMT>(x, __ldg(s + c * 8 + e), scale, rn)
-                                                    : exact_code_fmt<MODE, FMT>(x, __ldg(s + c * 8 + e), scale, rn));
+                if (redo && dchk(c < nchunks, SITE_DBG_RING_REPAIR)) {
+                    uint32_t code;
+                    if (FMT == kInt8 && !smooth) code = near_tie_code(vf, scale, __fmul_rn(vf, r));   // vf exact
+                    else if (second) code = exact_code_fmt<kSmooth, FMT>(x, __ldg(s + c * 8 + e), scale, rn);
+                    else code = exact_code_fmt<MODE, FMT>(x, __ldg(s + c * 8 + e), scale, rn);
+                    rq[c * 8 + e] = (int8_t)code;
+                }
             }
         }
     }
