@@ -433,12 +433,15 @@ __device__ __noinline__ uint32_t exact_code(float x, float s_j, float scale, flo
 }
 
 // The int8 code clamp(round_half_even(RN(v / scale)), -127, 127) of an exact
-// value v whose approximate quotient p (within 2^-15 of v / scale) lies within
-// 2^-13 of the half-integer h = floor(p) + 1/2, without a division. The true
-// quotient Q = v / scale is then within 2^-12 of h, so v - h * scale is a
-// multiple of 2^(e - 25) (e the exponent of scale; h a multiple of 1/2, v no
-// finer) below 2^(e - 11) in magnitude: exact in one fused multiply-add, and its
-// sign places Q against h. RN(Q) = h exactly when |Q - h| <= ulp(h) / 2, i.e.
+// value v whose true quotient Q = v / scale lies within 2^-12 of the
+// half-integer h = floor(p) + 1/2, p an approximate quotient, without a
+// division. (The callers pass p = RN(v * RN(1 / scale)), within 1.6e-5 of Q,
+// for elements whose fast quotient their near-tie test put within 2^-13 of h;
+// that fast quotient is within 3.8e-5 of Q, so |Q - h| <= 1.6e-4 < 2^-12.)
+// Then v - h * scale is a multiple of 2^(e - 25) (e the exponent of scale; h a
+// multiple of 1/2, v no finer) below 2^(e - 11) in magnitude: exact in one
+// fused multiply-add, and its sign places Q against h. RN(Q) = h exactly when
+// |Q - h| <= ulp(h) / 2, i.e.
 // when |v - h * scale| <= scale * ulp(h) / 2 (a product with a power of two,
 // exact); the equal case belongs to h because h, a multiple of 1/2 below 2^23,
 // has an even significand. A quotient that rounds to h takes h's even
@@ -550,8 +553,10 @@ __device__ __forceinline__ uint2 fix_near_ties_in(const RawChunk<T>& ch, uint2 c
         const float qv = __fmul_rn(ve, r);
         const float d = __fsub_rn(qv, __fsub_rn(__fadd_rn(qv, kMagic), kMagic));
         if (fabsf(d) >= 0.5f - kTieGuard) {
-            const uint32_t code = MODE == kSmooth ? exact_code<MODE>(ch.get(e), __ldg(s8 + e), scale, rn)
-                                                  : near_tie_code(ve, scale, qv);
+            // smooth: the exact value takes a division; its quotient stays
+            // within 2^-12 of the same half-step (v' is within 3 * 2^-24 |v| of v)
+            const float vx = MODE == kSmooth ? __fdiv_rn(ch.get(e), __ldg(s8 + e)) : ve;
+            const uint32_t code = near_tie_code(vx, scale, MODE == kSmooth ? __fmul_rn(vx, r) : qv);
             const int sh = 8 * (e & 3);
             uint32_t& w = (e < 4) ? codes.x : codes.y;
             w = (w & ~(0xffu << sh)) | (code << sh);
@@ -797,7 +802,9 @@ row_quant_fast_kernel(const T* __restrict__ in, int64_t rows, int64_t K, const f
 // maximum is always among them, since m' <= a(1 + 3 * 2^-24) and the element
 // attaining a has |v'| >= a(1 - 3 * 2^-24). (Resolving candidates against
 // each lane's own maximum instead saves the second group reduction but puts an
-// IEEE division in every lane: measured slower, 20.5 -> 22.5 us at K = 4096.)
+// IEEE division in every lane: measured slower, 20.5 -> 22.5 us at K = 4096;
+// against each warp's own maximum, one division per warp, it measured no
+// faster at K = 28672: fewer barrier waits, 15% more instructions.)
 //
 // Codes (pass 2): with r = RN(1/scale), t = RN(v * r + 1.5 * 2^23) holds
 // k = round-half-even(v * r) in its low mantissa bits, and d = RN(v * r - k)
@@ -1191,8 +1198,13 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                 }
                 if (redo && dchk(c < nchunks, SITE_DBG_RING_REPAIR)) {
                     uint32_t code;
-                    if (FMT == kInt8 && !smooth) code = near_tie_code(vf, scale, __fmul_rn(vf, r));   // vf exact
-                    else if (second) code = exact_code_fmt<kSmooth, FMT>(x, __ldg(s + c * 8 + e), scale, rn);
+                    if (FMT == kInt8) {
+                        // fold and norm: vf is exact; smooth: the exact value takes a
+                        // division, and its quotient stays within 2^-12 of the same
+                        // half-step (v' is within 3 * 2^-24 |v| of v)
+                        const float vx = smooth ? __fdiv_rn(x, __ldg(s + c * 8 + e)) : vf;
+                        code = near_tie_code(vx, scale, __fmul_rn(vx, r));
+                    } else if (second) code = exact_code_fmt<kSmooth, FMT>(x, __ldg(s + c * 8 + e), scale, rn);
                     else code = exact_code_fmt<MODE, FMT>(x, __ldg(s + c * 8 + e), scale, rn);
                     rq[c * 8 + e] = (int8_t)code;
                 }
