@@ -90,7 +90,7 @@ def _check_e4m3_gemm(y, xq, xs, wq, ws, out_dtype, what):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 300, 272), (5, 1024, 4096), (128, 512, 1040), (129, 257, 272),
-                                   (300, 1000, 2048), (1024, 768, 4096)])
+                                   (300, 1000, 2048), (1024, 768, 4096), (260, 1000, 16400)])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_e4m3_gemm_within_fp32_summation_bound(M, N, K, out_dtype):
     xq, wq, xs, ws = _codes(M, N, K, seed=M + N + K)

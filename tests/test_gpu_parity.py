@@ -198,6 +198,9 @@ GEMM_SHAPES = [
     (17, 256, 128), (100, 300, 272), (128, 256, 128), (129, 257, 144), (256, 512, 1024),
     (300, 1000, 2048), (1024, 768, 4096), (129, 4096, 1024), (513, 1000, 1040),
     (1024, 9728, 512), (777, 10000, 272), (2048, 12288, 1024),
+    # K >= 16384 and M > 128: the paired kernel's 512-column tiles (ragged N, K
+    # not a multiple of the 128-wide k-block, several tiles per pair)
+    (300, 1000, 16384), (257, 1536, 16400), (512, 1536, 28672),
 ]
 
 
@@ -210,7 +213,7 @@ def test_gemm_int32_exact(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (7, 300, 272), (16, 1024, 1024), (100, 300, 272),
-                                   (129, 257, 144), (512, 768, 1024)])
+                                   (129, 257, 144), (512, 768, 1024), (300, 1000, 16384)])
 def test_gemm_dequant_outputs(M, N, K):
     xq, wq, xs, wsc = _codes(M, N, K, seed=M + 7 * N + K)
     acc = oracle.gemm_i8(xq.numpy(), wq.numpy())

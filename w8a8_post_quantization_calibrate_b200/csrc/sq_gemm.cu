@@ -434,14 +434,23 @@ gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 // barrier arrival -- no data multicast). Each CTA's TMEM holds its 128 rows x
 // 256 columns of the accumulator (double-buffered); its epilogue warps drain
 // it and arrive on CTA 0's "accumulator empty" barrier.
-constexpr int P_STAGES = 6;
+//
+// Wide tiles (NT = 512 columns, for long K): each CTA loads two 128-row boxes
+// of B per stage (its halves of the tile's two 256-column blocks), CTA 0 issues
+// two N = 256 MMAs per k-step into TMEM columns 0..255 and 256..511, and the
+// single accumulator fills all 512 columns, so the epilogue of a tile is not
+// overlapped with the next tile's MMAs. Per k-step a pair moves 96 KB for
+// 256 x 512 outputs instead of 64 KB for 256 x 256: a quarter less operand
+// traffic per product through L2 and shared memory, and half as many tiles
+// re-reading the same panels from DRAM.
 constexpr uint32_t P_A_STAGE = 128 * BK;        // 16 KB: this CTA's 128 rows of A
-constexpr uint32_t P_B_STAGE = 128 * BK;        // 16 KB: this CTA's 128 rows of B
-constexpr uint32_t P_TX_BYTES = 2 * (P_A_STAGE + P_B_STAGE);   // both CTAs, per stage
 constexpr uint32_t IDESC_PAIR = make_idesc_i8(256, 256);
+__host__ __device__ constexpr int pair_stages(int nt) { return nt == 512 ? 4 : 6; }
+__host__ __device__ constexpr uint32_t pair_b_stage(int nt) { return (uint32_t)(nt / 2) * BK; }   // this CTA's rows of B
+__host__ __device__ constexpr int pair_accs(int nt) { return nt == 512 ? 1 : 2; }   // TMEM accumulators of nt columns
 
-constexpr size_t pair_smem_bytes() {
-    return 1024 + P_STAGES * (P_A_STAGE + P_B_STAGE) + 256;
+constexpr size_t pair_smem_bytes(int nt) {
+    return 1024 + (size_t)pair_stages(nt) * (P_A_STAGE + pair_b_stage(nt)) + 256;
 }
 
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cta0, int32_t x, int32_t y) {
@@ -505,11 +514,17 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "n"(NCOLS) : "memory");
 }
 
-template <int OUT, bool SPLIT, bool F8 = false>
+template <int OUT, bool SPLIT, bool F8 = false, int NT = 256>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ x_scale, const float* __restrict__ w_scale,
                  void* __restrict__ y, int M, int N, int K, const SplitTerm sp, long long wait_limit) {
+    static_assert(NT == 256 || NT == 512, "256- or 512-column tiles");
+    static_assert(NT == 256 || !SPLIT, "the outlier term's staging is sized for 256 columns");
+    constexpr int P_STAGES = pair_stages(NT);
+    constexpr uint32_t P_B_STAGE = pair_b_stage(NT);
+    constexpr uint32_t P_TX_BYTES = 2 * (P_A_STAGE + P_B_STAGE);   // both CTAs, per stage
+    constexpr int ACCS = pair_accs(NT);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -523,12 +538,21 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int num_m = (M + 255) / 256, num_n = (N + 255) / 256;
+    const int num_m = (M + 255) / 256, num_n = (N + NT - 1) / NT;
     const int num_tiles = num_m * num_n;
     const int num_kb = (K + BK - 1) / BK;
 
     auto bar = [&](int i) { return smem_u32(bars + i); };
     const int FULL = 0, EMPTY = P_STAGES, TFULL = 2 * P_STAGES, TEMPTY = 2 * P_STAGES + 2, DRAIN = 2 * P_STAGES + 4;
+    // the next accumulator and the parity of its barriers
+    auto next_acc = [](int& acc, uint32_t& acc_phase) {
+        if (ACCS == 2) {
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        } else {
+            acc_phase ^= 1;
+        }
+    };
     // entry 2 * P_STAGES + 5 holds the TMEM address and the abort flag
     const int SFULL = 2 * P_STAGES + 6, SEMPTY = 2 * P_STAGES + 7;   // this CTA's own staging
 
@@ -577,7 +601,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 int mb, nb;
                 tile_coords(tile, num_m, num_n, mb, nb);
                 const int arow = mb * 256 + (int)rank * 128;
-                const int brow = nb * 256 + (int)rank * 128;
+                const int brow = nb * NT + (int)rank * 128;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(bar(EMPTY + stage), phase ^ 1, wait_limit, abort_flag, SITE_GEMM_PRODUCER)) {
                         ok = false;
@@ -587,6 +611,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     if (rank == 0) mbar_arrive_expect_tx(bar(FULL + stage), P_TX_BYTES);
                     tma_load_2d_pair(smem_u32(sA + stage * P_A_STAGE), &tmA, full0, kb * BK, arow);
                     tma_load_2d_pair(smem_u32(sB + stage * P_B_STAGE), &tmB, full0, kb * BK, brow);
+                    if (NT == 512)   // this CTA's half of the second 256-column block
+                        tma_load_2d_pair(smem_u32(sB + stage * P_B_STAGE + 128 * BK), &tmB, full0, kb * BK, brow + 256);
                     ++issued;
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -617,7 +643,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
                 if (!mbar_wait(bar(TEMPTY + acc), acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM_MMA_TMEM)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NT);
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(bar(FULL + stage), phase, wait_limit, abort_flag, SITE_GEMM_MMA_FULL)) {
                         ok = false;
@@ -627,16 +653,19 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const uint32_t a0 = smem_u32(sA + stage * P_A_STAGE);
                     const uint32_t b0 = smem_u32(sB + stage * P_B_STAGE);
 #pragma unroll
-                    for (int k = 0; k < BK / UMMA_K; ++k)
-                        mma_pair<F8>(d_tmem, make_sw128_kmajor_desc(a0 + k * UMMA_K),
-                                     make_sw128_kmajor_desc(b0 + k * UMMA_K), (kb | k) != 0 ? 1u : 0u);
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        const uint64_t ad = make_sw128_kmajor_desc(a0 + k * UMMA_K);
+                        mma_pair<F8>(d_tmem, ad, make_sw128_kmajor_desc(b0 + k * UMMA_K), (kb | k) != 0 ? 1u : 0u);
+                        if (NT == 512)
+                            mma_pair<F8>(d_tmem + 256, ad, make_sw128_kmajor_desc(b0 + 128 * BK + k * UMMA_K),
+                                         (kb | k) != 0 ? 1u : 0u);
+                    }
                     mma_commit_pair(bar(EMPTY + stage));
                     if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
                 mma_commit_pair(bar(TFULL + acc));
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1;
+                next_acc(acc, acc_phase);
             }
             mma_commit_cta0(bar(DRAIN));
             mbar_wait(bar(DRAIN), 0, wait_limit, &no_abort, SITE_GEMM_DRAIN);
@@ -658,14 +687,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const int64_t row = (int64_t)mb * 256 + rank * 128 + quarter * 32 + lane;
             const bool row_ok = row < M;
             const float sa = (OUT != kOutI32 && row_ok) ? __ldg(x_scale + row) : 0.0f;
-            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NT);
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; c += 2) {
+            for (int c = 0; c < NT / 32; c += 2) {
                 uint32_t r0[32], r1[32];
                 tmem_ld_32x32b_x32(taddr + c * 32, r0);
                 tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
                 tmem_wait_ld();
-                const int col0 = nb * BN + c * 32;
+                const int col0 = nb * NT + c * 32;
                 const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
                 if (row_ok && col0 < N)
                     store_row32<OUT, SPLIT, F8 ? kAkE4M3 : kAkI8>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
@@ -679,8 +708,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 else arrive_on_cta0(bar(TEMPTY + acc));
                 if (SPLIT) mbar_arrive(bar(SEMPTY));   // this warp has read the staged tile
             }
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1;
+            next_acc(acc, acc_phase);
         }
     }
 
@@ -1247,19 +1275,32 @@ sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float
                       ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
 }
 
+template <int OUT, bool SPLIT, bool F8, int NT>
+sq_status launch_pair_nt(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
+                         int M, int N, int K, cudaStream_t st, const SplitTerm& sp) {
+    static bool attr_done[64] = {};
+    const DeviceInfo& di = device_info();
+    const size_t smem = pair_smem_bytes(NT) + (SPLIT ? kSplitSmem : 0);
+    sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT, SPLIT, F8, NT>, smem, attr_done[di.device & 63]);
+    if (r != SQ_OK) return r;
+    const int tiles = ((M + 255) / 256) * ((N + NT - 1) / NT);
+    const int max_pairs = di.sm_count / 2;
+    const int pairs = tiles < max_pairs ? tiles : max_pairs;
+    return launch_pdl("gemm_pair_kernel", gemm_pair_kernel<OUT, SPLIT, F8, NT>, dim3(2 * pairs), dim3(GEMM_THREADS),
+                      smem, st, 2, ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
+}
+
+// Wide (512-column) tiles for long K, where a tile's main loop dwarfs its
+// unoverlapped epilogue; 256-column tiles otherwise and for the outlier term.
+constexpr int kWidePairMinK = 16384;
+
 template <int OUT, bool SPLIT = false, bool F8 = false>
 sq_status launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
                       int M, int N, int K, cudaStream_t st, const SplitTerm& sp = SplitTerm{}) {
-    static bool attr_done[64] = {};
-    const DeviceInfo& di = device_info();
-    const size_t smem = pair_smem_bytes() + (SPLIT ? kSplitSmem : 0);
-    sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT, SPLIT, F8>, smem, attr_done[di.device & 63]);
-    if (r != SQ_OK) return r;
-    const int tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    const int max_pairs = di.sm_count / 2;
-    const int pairs = tiles < max_pairs ? tiles : max_pairs;
-    return launch_pdl("gemm_pair_kernel", gemm_pair_kernel<OUT, SPLIT, F8>, dim3(2 * pairs), dim3(GEMM_THREADS), smem, st,
-                      2, ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
+    if constexpr (!SPLIT) {
+        if (K >= kWidePairMinK) return launch_pair_nt<OUT, SPLIT, F8, 512>(ta, tb, xs, wsc, y, M, N, K, st, sp);
+    }
+    return launch_pair_nt<OUT, SPLIT, F8, 256>(ta, tb, xs, wsc, y, M, N, K, st, sp);
 }
 
 template <int OUT, bool SPLIT = false>
