@@ -448,10 +448,6 @@ constexpr uint32_t IDESC_PAIR = make_idesc_i8(256, 256);
 __host__ __device__ constexpr int pair_stages(int nt) { return nt == 512 ? 4 : 6; }
 __host__ __device__ constexpr uint32_t pair_b_stage(int nt) { return (uint32_t)(nt / 2) * BK; }   // this CTA's rows of B
 __host__ __device__ constexpr int pair_accs(int nt) { return nt == 512 ? 1 : 2; }   // TMEM accumulators of nt columns
-// Threads of a pair CTA: warp 0 TMA, warp 1 MMA, then the epilogue warps, one
-// per TMEM lane quarter and 256 columns (wide tiles: two per quarter, halving
-// the epilogue the main loop cannot hide).
-__host__ __device__ constexpr int pair_threads(int nt) { return nt == 512 ? 320 : 192; }
 
 constexpr size_t pair_smem_bytes(int nt) {
     return 1024 + (size_t)pair_stages(nt) * (P_A_STAGE + pair_b_stage(nt)) + 256;
@@ -519,7 +515,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr) {
 }
 
 template <int OUT, bool SPLIT, bool F8 = false, int NT = 256>
-__global__ void __launch_bounds__(pair_threads(NT), 1)
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ x_scale, const float* __restrict__ w_scale,
                  void* __restrict__ y, int M, int N, int K, const SplitTerm sp, long long wait_limit) {
@@ -529,7 +525,6 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     constexpr uint32_t P_B_STAGE = pair_b_stage(NT);
     constexpr uint32_t P_TX_BYTES = 2 * (P_A_STAGE + P_B_STAGE);   // both CTAs, per stage
     constexpr int ACCS = pair_accs(NT);
-    constexpr int EPI_WARPS = pair_threads(NT) / 32 - 2;   // 4 or 8; warp w reads TMEM lane quarter w % 4
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -568,7 +563,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(bar(TFULL + a), 1);
-            mbar_init(bar(TEMPTY + a), 2 * EPI_WARPS);   // every epilogue warp of both CTAs
+            mbar_init(bar(TEMPTY + a), 8);   // 4 epilogue warps in each CTA
         }
         mbar_init(bar(DRAIN), 1);
         if (SPLIT) {
@@ -677,9 +672,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------- epilogue (warps 2.., both CTAs)
+        // ---------------------------------------------------- epilogue (warps 2..5, both CTAs)
         const int quarter = warp & 3;
-        const int cgroup = (warp - 2) >> 2;   // its 256 columns of the tile
         int acc = 0;
         uint32_t acc_phase = 0;
         float* w_s = reinterpret_cast<float*>(smem + P_STAGES * (P_A_STAGE + P_B_STAGE) + 256);
@@ -695,7 +689,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const float sa = (OUT != kOutI32 && row_ok) ? __ldg(x_scale + row) : 0.0f;
             const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NT);
 #pragma unroll 1
-            for (int c = cgroup * 8; c < cgroup * 8 + 8; c += 2) {
+            for (int c = 0; c < NT / 32; c += 2) {
                 uint32_t r0[32], r1[32];
                 tmem_ld_32x32b_x32(taddr + c * 32, r0);
                 tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
@@ -1292,8 +1286,8 @@ sq_status launch_pair_nt(const CUtensorMap& ta, const CUtensorMap& tb, const flo
     const int tiles = ((M + 255) / 256) * ((N + NT - 1) / NT);
     const int max_pairs = di.sm_count / 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
-    return launch_pdl("gemm_pair_kernel", gemm_pair_kernel<OUT, SPLIT, F8, NT>, dim3(2 * pairs),
-                      dim3(pair_threads(NT)), smem, st, 2, ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
+    return launch_pdl("gemm_pair_kernel", gemm_pair_kernel<OUT, SPLIT, F8, NT>, dim3(2 * pairs), dim3(GEMM_THREADS),
+                      smem, st, 2, ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
 }
 
 // Wide (512-column) tiles for long K, where a tile's main loop dwarfs its
