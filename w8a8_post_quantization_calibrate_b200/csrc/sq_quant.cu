@@ -820,6 +820,23 @@ constexpr int kRingThreads = 512;
 constexpr int kRingCPL = 8;
 constexpr size_t kRingSmemMax = 231424;   // dynamic shared memory of one CTA (226 KB of the 227 KB opt-in)
 constexpr float kRingCandidate = 1.0f - 1.0f / 1048576.0f;
+// Near-tie guards of the streamed kernel. Its fast quotient is v' * r taken
+// exactly inside the fused multiply-add (r = RN(1/scale)); against q* = RN(v /
+// scale), |q| <= 127.5:
+//   |v' r - q*| <= |v' - v| r + |v| |r - 1/scale| + ulp(q*) / 2
+//              <= 3 * 2^-24 * 127.5 + 2^-24 * 127.5 + 2^-18 = 3.4e-5  (smooth: v' within 3 * 2^-24 |v|)
+//              <= 2^-24 * 127.5 + 2^-18 = 1.2e-5                      (fold, norm: v exact)
+// An element farther than the guard from a half-step has q* on the same side.
+constexpr float kRingGuardExact = 1.0f / 32768.0f;    // 3.05e-5
+constexpr float kRingGuardSmooth = 1.0f / 16384.0f;   // 6.1e-5
+
+// Bring the 128-byte line holding p into L1 ahead of a load on a rare path
+// (the smoothing kernel's near-tie repair reads s_j, which no shared-memory
+// table holds; the same prefetch for the maximum's candidates, issued before the
+// group reduction, measured slower: 190 -> 225 us at K = 28672).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+    asm volatile("{\n\t.reg .u64 a;\n\tcvta.to.global.u64 a, %0;\n\tprefetch.global.L1 [a];\n\t}" :: "l"(p));
+}
 
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -1116,6 +1133,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         const float scale = __fdiv_rn(amax, kQmax);
         const float r = __frcp_rn(scale);
         const uint64_t r2 = f2_pack(r, r);
+        const float guard = smooth ? kRingGuardSmooth : kRingGuardExact;
         uint32_t ntm = 0;
         uint2 codes[CPL];
         if constexpr (FMT == kInt8) {
@@ -1136,7 +1154,9 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                 }
                 codes[i].x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
                 codes[i].y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
-                ntm |= (dm >= 0.5f - kTieGuard ? 1u : 0u) << i;   // (padding: d = 0)
+                const bool tie = dm >= 0.5f - guard;   // (padding: d = 0)
+                if (smooth && tie) prefetch_l1(s + (gl + i * 32 * R) * 8);   // the repair divides by s_j
+                ntm |= (tie ? 1u : 0u) << i;
             }
         } else {
             // E4M3: q' = RN(v r) converted at q'(1 - 2^-18) and q'(1 + 2^-18);
@@ -1190,7 +1210,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                 if (FMT == kInt8) {
                     const float tf = __fmaf_rn(vf, r, kMagic);
                     const float df = __fmaf_rn(vf, r, __fsub_rn(kMagic, tf));
-                    redo = fabsf(df) >= 0.5f - kTieGuard;
+                    redo = fabsf(df) >= 0.5f - guard;
                 } else {
                     const float qf = __fmul_rn(vf, r);
                     redo = __nv_cvt_float_to_fp8(__fmul_rn(qf, 1.0f - 1.0f / 262144.0f), __NV_SATFINITE, __NV_E4M3) !=
