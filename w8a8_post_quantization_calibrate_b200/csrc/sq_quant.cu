@@ -981,6 +981,19 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
     int it = 0, sl = 0, ps = ns - 1;   // iteration, its slot, the previous iteration's slot
     uint32_t parity = 0;
     bool failed = false;
+    // One smoothing near-tie per lane is carried to the next row: its s_j load
+    // (global memory; no shared-memory table holds s_j) is issued when the tie
+    // is found and consumed a row later, off the group's barrier path.
+    bool pend = false;
+    float pend_x = 0.0f, pend_s = 1.0f, pend_scale = 1.0f, pend_r = 1.0f;
+    int8_t* pend_q = nullptr;
+    auto settle = [&]() {
+        if (FMT == kInt8 && pend) {
+            const float vx = __fdiv_rn(pend_x, pend_s);
+            *pend_q = (int8_t)near_tie_code(vx, pend_scale, __fmul_rn(vx, pend_r));
+            pend = false;
+        }
+    };
     for (int64_t g = row0; g < total; g += stride, ++it) {
         // this row's tensor: the first (MODE), or the second (smoothed) of a pair
         const bool second = PAIR && g >= rows;
@@ -1057,6 +1070,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
             cm[i] = cmax;
             m = fmaxf(m, cmax);
         }
+        settle();   // the previous row's carried repair, its load long done
         float amax = group_max<R>(m, red, grp, wig, lane, bank);
         bank ^= 1;
         int8_t* rq = qo + row * K;
@@ -1222,6 +1236,15 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
                         // fold and norm: vf is exact; smooth: the exact value takes a
                         // division, and its quotient stays within 2^-12 of the same
                         // half-step (v' is within 3 * 2^-24 |v| of v)
+                        if (smooth && !pend) {
+                            pend = true;
+                            pend_x = x;
+                            pend_s = __ldg(s + c * 8 + e);
+                            pend_scale = scale;
+                            pend_r = r;
+                            pend_q = rq + c * 8 + e;
+                            continue;
+                        }
                         const float vx = smooth ? __fdiv_rn(x, __ldg(s + c * 8 + e)) : vf;
                         code = near_tie_code(vx, scale, __fmul_rn(vx, r));
                     } else if (second) code = exact_code_fmt<kSmooth, FMT>(x, __ldg(s + c * 8 + e), scale, rn);
@@ -1232,6 +1255,7 @@ row_quant_ring_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_
         }
     }
 
+    settle();
     if (failed && gl == 0) {
         // copies issued for rows this group will not consume: let them land
         // before the CTA exits (bounded)
