@@ -134,6 +134,26 @@ def test_near_ties(K):
     check_smooth(torch.ones(2, K, dtype=BF16), s_smooth, f"smooth near ties K={K}")
 
 
+@pytest.mark.parametrize("K", [4096, 28672])
+def test_near_ties_in_every_row(K):
+    """Hundreds of smoothing near-ties in each of 600 rows (rows 2^k x, which
+    keeps every quotient): a lane carries its first tie of a row to the next row
+    and repairs the rest at once, across the several rows each CTA works."""
+    scale = np.float32(30.0) / np.float32(127.0)
+    t = _tie_targets(scale)
+    rng = np.random.default_rng(K + 11)
+    pos = rng.permutation(np.arange(1, K))[: len(t)]
+    s_fold = rng.uniform(0.01, 0.2, K).astype(np.float32)
+    s_fold[0] = 30.0
+    s_fold[pos] = t
+    s_smooth = (np.float32(1.0) / s_fold).astype(np.float32)
+    k = torch.from_numpy(rng.integers(-6, 7, 600).astype(np.float32))
+    x = (torch.ones(600, K) * torch.pow(2.0, k)[:, None]).to(BF16)
+    x[::7] = -x[::7]
+    check_smooth(x, s_smooth, f"smooth near ties in every row K={K}")
+    check_fold(x, s_fold, f"fold near ties in every row K={K}")
+
+
 @pytest.mark.parametrize("K", [4096, 5120, 6160, 16384])
 def test_many_candidates_for_the_maximum(K):
     """Smoothed rows whose largest values differ by a few ulps, spread over
