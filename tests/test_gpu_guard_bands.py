@@ -21,7 +21,9 @@ if not torch.cuda.is_available():
 from w8a8_post_quantization_calibrate_b200 import sq  # noqa: E402
 
 DEV = torch.device("cuda", 0)
-SHAPES = [(1, 3, 16), (5, 7, 48), (13, 129, 1040), (130, 257, 2064), (17, 300, 5136), (3, 5, 28672)]
+# (260, 600, 16400): the paired GEMM's 512-column tiles, N and K ragged
+SHAPES = [(1, 3, 16), (5, 7, 48), (13, 129, 1040), (130, 257, 2064), (17, 300, 5136), (3, 5, 28672),
+          (260, 600, 16400)]
 
 
 def _xw(T, N, K, dtype, seed):
@@ -73,7 +75,7 @@ def test_steps_stay_inside_their_outputs(dtype, T, N, K):
     assert sq.sq_get_status() == sq.SQ_OK
 
 
-@pytest.mark.parametrize("T,N,K", [(1, 3, 16), (5, 7, 48), (16, 300, 1040), (200, 257, 2064)])
+@pytest.mark.parametrize("T,N,K", [(1, 3, 16), (5, 7, 48), (16, 300, 1040), (200, 257, 2064), (260, 600, 16384)])
 def test_variants_stay_inside_their_outputs(T, N, K):
     x, w = _xw(T, N, K, torch.bfloat16, seed=T + N + K)
     xd, wd = x.to(DEV), w.to(DEV)
