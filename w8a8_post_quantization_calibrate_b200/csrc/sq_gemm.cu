@@ -178,7 +178,8 @@ __device__ __forceinline__ float add_split1(float v, int64_t t, int64_t n, const
 
 // Stores 32 consecutive outputs of one row (row-major y, row stride N). For
 // bf16 operands (AK == kAkBF16) the outputs are the raw fp32 accumulators.
-template <int OUT, bool SPLIT, int AK = kAkI8>
+// SW_SMEM: w_scale points into a shared-memory copy (read with plain loads).
+template <int OUT, bool SPLIT, int AK = kAkI8, bool SW_SMEM = false>
 __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int N, const uint32_t (&r)[32],
                                             float sa, const float* __restrict__ w_scale, const float* xr,
                                             const float* ws_col, int ld) {
@@ -204,7 +205,8 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
     } else if (full) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
-            const float4 sw = __ldg(reinterpret_cast<const float4*>(w_scale + col0 + i));
+            const float4 sw = SW_SMEM ? *reinterpret_cast<const float4*>(w_scale + col0 + i)
+                                      : __ldg(reinterpret_cast<const float4*>(w_scale + col0 + i));
             v[i] = dequant_raw<F8>(r[i], sa, sw.x);
             v[i + 1] = dequant_raw<F8>(r[i + 1], sa, sw.y);
             v[i + 2] = dequant_raw<F8>(r[i + 2], sa, sw.z);
@@ -213,7 +215,8 @@ __device__ __forceinline__ void store_row32(void* y, int64_t row, int col0, int 
     } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-            v[i] = (col0 + i < N) ? dequant_raw<F8>(r[i], sa, __ldg(w_scale + col0 + i)) : 0.0f;
+            v[i] = (col0 + i < N) ? dequant_raw<F8>(r[i], sa, SW_SMEM ? w_scale[col0 + i] : __ldg(w_scale + col0 + i))
+                                  : 0.0f;
     }
     if (SPLIT) add_split32(v, xr, ws_col, ld);
     if (OUT == kOutF32) {
@@ -452,6 +455,11 @@ __host__ __device__ constexpr int pair_accs(int nt) { return nt == 512 ? 1 : 2; 
 constexpr size_t pair_smem_bytes(int nt) {
     return 1024 + (size_t)pair_stages(nt) * (P_A_STAGE + pair_b_stage(nt)) + 256;
 }
+// Beyond the ring: the outlier term's staging (SPLIT), or else one copy per
+// epilogue warp of the tile's output-channel scales.
+constexpr size_t pair_epilogue_smem_bytes(int nt, bool split) {
+    return split ? kSplitSmem : 4 * (size_t)nt * sizeof(float);
+}
 
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cta0, int32_t x, int32_t y) {
     asm volatile(
@@ -677,10 +685,30 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         int acc = 0;
         uint32_t acc_phase = 0;
         float* w_s = reinterpret_cast<float*>(smem + P_STAGES * (P_A_STAGE + P_B_STAGE) + 256);
+        // without the outlier term: this warp's copy of the tile's output-channel
+        // scales, loaded while the tile's main loop runs (the warp is done with
+        // the previous tile), so the epilogue reads them from shared memory
+        float* scl = w_s + (warp - 2) * NT;
         uint32_t it = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
             int mb, nb;
             tile_coords(tile, num_m, num_n, mb, nb);
+            if (!SPLIT && OUT != kOutI32) {
+#pragma unroll
+                for (int i = lane * 4; i < NT; i += 128) {
+                    const int col = nb * NT + i;
+                    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    if (col + 3 < N) {
+                        v = __ldg(reinterpret_cast<const float4*>(w_scale + col));
+                    } else {
+                        if (col < N) v.x = __ldg(w_scale + col);
+                        if (col + 1 < N) v.y = __ldg(w_scale + col + 1);
+                        if (col + 2 < N) v.z = __ldg(w_scale + col + 2);
+                    }
+                    *reinterpret_cast<float4*>(scl + i) = v;
+                }
+                __syncwarp();
+            }
             if (SPLIT && !stage_split(w_s, sp, nb, N, it, bar(SFULL), bar(SEMPTY), wait_limit, abort_flag)) break;
             if (!mbar_wait(bar(TFULL + acc), acc_phase, wait_limit, abort_flag, SITE_GEMM_EPILOGUE)) break;
             tc_fence_after();
@@ -696,10 +724,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tmem_wait_ld();
                 const int col0 = nb * NT + c * 32;
                 const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
+                // scales indexed by absolute column: this warp's copy, or global memory
+                const float* sw_base = SPLIT ? w_scale : scl - nb * NT;
                 if (row_ok && col0 < N)
-                    store_row32<OUT, SPLIT, F8 ? kAkE4M3 : kAkI8>(y, row, col0, N, r0, sa, w_scale, xr, w_s + c * 32, sp.ld);
+                    store_row32<OUT, SPLIT, F8 ? kAkE4M3 : kAkI8, !SPLIT>(y, row, col0, N, r0, sa, sw_base, xr,
+                                                                          w_s + c * 32, sp.ld);
                 if (row_ok && col0 + 32 < N)
-                    store_row32<OUT, SPLIT, F8 ? kAkE4M3 : kAkI8>(y, row, col0 + 32, N, r1, sa, w_scale, xr, w_s + (c + 1) * 32, sp.ld);
+                    store_row32<OUT, SPLIT, F8 ? kAkE4M3 : kAkI8, !SPLIT>(y, row, col0 + 32, N, r1, sa, sw_base, xr,
+                                                                          w_s + (c + 1) * 32, sp.ld);
             }
             tc_fence_before();
             __syncwarp();
@@ -1280,7 +1312,7 @@ sq_status launch_pair_nt(const CUtensorMap& ta, const CUtensorMap& tb, const flo
                          int M, int N, int K, cudaStream_t st, const SplitTerm& sp) {
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
-    const size_t smem = pair_smem_bytes(NT) + (SPLIT ? kSplitSmem : 0);
+    const size_t smem = pair_smem_bytes(NT) + pair_epilogue_smem_bytes(NT, SPLIT);
     sq_status r = ensure_smem_attr(gemm_pair_kernel<OUT, SPLIT, F8, NT>, smem, attr_done[di.device & 63]);
     if (r != SQ_OK) return r;
     const int tiles = ((M + 255) / 256) * ((N + NT - 1) / NT);
