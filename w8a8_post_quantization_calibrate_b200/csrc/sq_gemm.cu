@@ -456,9 +456,12 @@ constexpr size_t pair_smem_bytes(int nt) {
     return 1024 + (size_t)pair_stages(nt) * (P_A_STAGE + pair_b_stage(nt)) + 256;
 }
 // Beyond the ring: the outlier term's staging (SPLIT), or else one copy per
-// epilogue warp of the tile's output-channel scales.
+// epilogue warp of the tile's output-channel scales and two 2 KB buffers per
+// epilogue warp for bf16 output blocks (32 rows x 32 columns) on their way to
+// global memory by bulk tensor stores.
+constexpr uint32_t kOutBlockBytes = 32 * 32 * 2;
 constexpr size_t pair_epilogue_smem_bytes(int nt, bool split) {
-    return split ? kSplitSmem : 4 * (size_t)nt * sizeof(float);
+    return split ? kSplitSmem : 4 * (size_t)nt * sizeof(float) + 4 * 2 * (size_t)kOutBlockBytes;
 }
 
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cta0, int32_t x, int32_t y) {
@@ -511,6 +514,17 @@ __device__ __forceinline__ void arrive_on_cta0(uint32_t local_bar) {
                  "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
                  :: "r"(local_bar) : "memory");
 }
+// Bulk tensor stores from shared memory (no multicast): issue, group, and wait
+// until a group no longer reads its source (or has completed).
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 :: "l"(tmap), "r"(src), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 template <int NCOLS>
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t holder_smem) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -526,7 +540,8 @@ template <int OUT, bool SPLIT, bool F8 = false, int NT = 256>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ x_scale, const float* __restrict__ w_scale,
-                 void* __restrict__ y, int M, int N, int K, const SplitTerm sp, long long wait_limit) {
+                 void* __restrict__ y, int M, int N, int K, const SplitTerm sp, long long wait_limit,
+                 const __grid_constant__ CUtensorMap tmY, int tstore) {
     static_assert(NT == 256 || NT == 512, "256- or 512-column tiles");
     static_assert(NT == 256 || !SPLIT, "the outlier term's staging is sized for 256 columns");
     constexpr int P_STAGES = pair_stages(NT);
@@ -689,6 +704,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // scales, loaded while the tile's main loop runs (the warp is done with
         // the previous tile), so the epilogue reads them from shared memory
         float* scl = w_s + (warp - 2) * NT;
+        // bf16 output by bulk tensor stores (tstore): the warp writes each 32 x 32
+        // block of its rows into one of its two buffers, and one lane stores it;
+        // the TMEM accumulator is released as soon as it has been read, and the
+        // stores drain while the next tile's MMAs run
+        const bool tma_out = OUT == kOutBF16 && !SPLIT && tstore != 0;
+        uint8_t* obuf = reinterpret_cast<uint8_t*>(w_s + 4 * NT) + (size_t)(warp - 2) * 2 * kOutBlockBytes;
+        uint32_t nblk = 0;
         uint32_t it = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
             int mb, nb;
@@ -723,6 +745,35 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
                 tmem_wait_ld();
                 const int col0 = nb * NT + c * 32;
+                if (tma_out) {
+                    const int row_w = mb * 256 + (int)rank * 128 + quarter * 32;   // the warp's first row
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const uint32_t* rr = j ? r1 : r0;
+                        const int cc = col0 + 32 * j;
+                        uint8_t* buf = obuf + (nblk & 1u) * kOutBlockBytes;
+                        if (lane == 0) bulk_wait_read_le1();   // this buffer's last store has read it
+                        __syncwarp();
+                        const float* sw = scl + (cc - nb * NT);   // zero past N
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2)
+                            pk[i / 2] = pack_bf16x2(dequant_raw<F8>(rr[i], sa, sw[i]),
+                                                    dequant_raw<F8>(rr[i + 1], sa, sw[i + 1]));
+                        uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0 && cc < N && row_w < M) {
+                            tma_store_2d(&tmY, smem_u32(buf), cc, row_w);   // rows past M, columns past N clipped
+                            bulk_commit_group();
+                        }
+                        ++nblk;
+                    }
+                    continue;
+                }
                 const float* xr = SPLIT && row_ok ? sp.x_out + row * sp.ld : nullptr;
                 // scales indexed by absolute column: this warp's copy, or global memory
                 const float* sw_base = SPLIT ? w_scale : scl - nb * NT;
@@ -742,6 +793,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             }
             next_acc(acc, acc_phase);
         }
+        if (tma_out && lane == 0) bulk_wait_all();   // every output block written
     }
 
     // neither CTA leaves while the other may still touch its shared memory or TMEM
@@ -1261,6 +1313,27 @@ sq_status make_map_i8(CUtensorMap* map, const void* base, int64_t rows, int64_t 
     return SQ_OK;
 }
 
+// Row-major bf16 output Y [M x N] as a 2-D tensor map for bulk stores of 32 x 32
+// blocks (no swizzle; out-of-range rows and columns are not written). N * 2
+// must be a multiple of 16 bytes.
+sq_status make_map_out_bf16(CUtensorMap* map, void* base, int64_t M, int64_t N) {
+    sq_status r = get_encoder();
+    if (r != SQ_OK) return r;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult cr = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d) for a %lld x %lld bf16 output", (int)cr, (long long)M,
+                  (long long)N);
+        return SQ_ERR_CUDA;
+    }
+    return SQ_OK;
+}
+
 // Row-major bf16 matrix [rows x K] as a 2-D tensor map with 128B swizzle and a
 // (64 elements = 128 bytes of K) x box_rows box.
 sq_status make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
@@ -1310,6 +1383,15 @@ sq_status launch_tiled(const CUtensorMap& ta, const CUtensorMap& tb, const float
 template <int OUT, bool SPLIT, bool F8, int NT>
 sq_status launch_pair_nt(const CUtensorMap& ta, const CUtensorMap& tb, const float* xs, const float* wsc, void* y,
                          int M, int N, int K, cudaStream_t st, const SplitTerm& sp) {
+    // bf16 output through bulk tensor stores where the row stride allows a map
+    CUtensorMap ty;
+    std::memset(&ty, 0, sizeof(ty));
+    int tstore = 0;
+    if (OUT == kOutBF16 && !SPLIT && (N % 8) == 0) {
+        sq_status rm = make_map_out_bf16(&ty, y, M, N);
+        if (rm != SQ_OK) return rm;
+        tstore = 1;
+    }
     static bool attr_done[64] = {};
     const DeviceInfo& di = device_info();
     const size_t smem = pair_smem_bytes(NT) + pair_epilogue_smem_bytes(NT, SPLIT);
@@ -1319,7 +1401,7 @@ sq_status launch_pair_nt(const CUtensorMap& ta, const CUtensorMap& tb, const flo
     const int max_pairs = di.sm_count / 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
     return launch_pdl("gemm_pair_kernel", gemm_pair_kernel<OUT, SPLIT, F8, NT>, dim3(2 * pairs), dim3(GEMM_THREADS),
-                      smem, st, 2, ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles());
+                      smem, st, 2, ta, tb, xs, wsc, y, M, N, K, sp, wait_limit_cycles(), ty, tstore);
 }
 
 // Wide (512-column) tiles for long K, where a tile's main loop dwarfs its
