@@ -199,8 +199,9 @@ GEMM_SHAPES = [
     (300, 1000, 2048), (1024, 768, 4096), (129, 4096, 1024), (513, 1000, 1040),
     (1024, 9728, 512), (777, 10000, 272), (2048, 12288, 1024),
     # K >= 16384 and M > 128: the paired kernel's 512-column tiles (ragged N, K
-    # not a multiple of the 128-wide k-block, several tiles per pair)
-    (300, 1000, 16384), (257, 1536, 16400), (512, 1536, 28672),
+    # not a multiple of the 128-wide k-block, several tiles per pair); just
+    # below that K, 256-column tiles
+    (300, 1000, 16384), (257, 1536, 16400), (512, 1536, 28672), (300, 1000, 16368),
 ]
 
 

@@ -104,6 +104,24 @@ def test_norm_stream(rows, K):
     check_norm(x, oracle.fold_norm_gain(gain, s_for(K, K + 7)), 1e-6, f"norm {rows}x{K}")
 
 
+# K (a multiple of 16, as the calls require) on either side of the streamed
+# kernel's range (2064..28672 channels): the calls pick a kernel by K, and each
+# side of each edge must match the oracle
+EDGE_K = [2032, 2048, 2064, 2080, 28656, 28672, 28688, 28704]
+
+
+@pytest.mark.parametrize("K", EDGE_K)
+def test_kernel_choice_edges(K):
+    rows = 7
+    g = torch.Generator().manual_seed(K + 11)
+    w = (torch.randn(rows, K, generator=g) * 0.05).to(BF16)
+    w[3] = 0
+    check_fold(w, s_for(K, K + 2), f"fold {rows}x{K}")
+    x = outlier_x(rows, K, seed=K + 13)
+    x[4, K // 5:] = 0
+    check_smooth(x, s_for(K, K + 3), f"smooth {rows}x{K}")
+
+
 def _tie_targets(scale):
     """fp32 values a few ulps either side of (k + 1/2) * scale, k = 0..126."""
     out = []
