@@ -24,7 +24,9 @@ if not torch.cuda.is_available():
 from w8a8_post_quantization_calibrate_b200 import sq  # noqa: E402
 
 DEV = torch.device("cuda", 0)
-ROW_SHAPES = [(1, 16), (5, 48), (130, 1040), (64, 4096), (9, 11008), (3, 28672), (2, 65536)]
+# (2048, 2064) and (28672, 28688): either side of the streamed kernel's K range
+ROW_SHAPES = [(1, 16), (5, 48), (130, 1040), (4, 2048), (4, 2064), (64, 4096), (9, 11008), (3, 28672),
+              (3, 28688), (2, 65536)]
 
 
 def dev(t):
